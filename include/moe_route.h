@@ -1,0 +1,223 @@
+/*
+ * moe_route.h -- C ABI of libmoeroute.so, the B200 (sm_100a) MoE routing hot
+ * path: gate GEMM + score nonlinearity, bias-adjusted group-limited top-K with
+ * combine weights, load histogram and statistics, bias update, and the
+ * expert-contiguous dispatch / weighted combine permutation.
+ *
+ * Conventions for every call
+ *  - All array arguments are DEVICE pointers to dense row-major arrays owned
+ *    by the caller.  The library never allocates, frees or synchronises; every
+ *    call only enqueues kernels on `stream` and returns.  Results are ready
+ *    when the stream reaches them.
+ *  - Arguments are validated on the host before any launch; a bad argument
+ *    returns MOE_ERR_INVALID (or MOE_ERR_UNSUPPORTED for a valid shape this
+ *    build has no kernel for) and enqueues nothing.  A failed launch returns
+ *    MOE_ERR_CUDA.  Nothing aborts or traps.
+ *  - Device-side waits (TMA/MMA barriers in the gate GEMM, the look-back of
+ *    the offsets scan) are bounded.  A wait that runs out sets an error word
+ *    in the workspace and the kernel returns early; read it with
+ *    moe_workspace_status().  The load-statistics struct also carries the
+ *    scan's status of that call.
+ *  - 16-byte alignment is required for x, w_gate, rows, y and out.
+ *  - Flat assignment counts must satisfy T*K < 2^31.
+ *
+ * Sources (web pages on MoE load balancing), cited per call below:
+ *  [ENT] "MoE Routing Entropy vs Expert Saturation: Optimizing DeepSeek V4
+ *        Load Balancing" (dailyaiworld.com)
+ *  [HD]  "DeepSeek V4 MoE load balancing" (blog.hotdry.top)
+ *  [GL]  "DeepSeek-V3 Group-Limited Expert Routing" (cnnetsun.cn)
+ *  [MIN] "A minimal experiment in expert-load imbalance" (tech-blog-chi)
+ */
+#ifndef MOE_ROUTE_H_
+#define MOE_ROUTE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID = 1,     /* bad argument; nothing enqueued */
+    MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented for this shape / dtype */
+    MOE_ERR_CUDA = 3,        /* a CUDA call failed */
+    MOE_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out */
+} moe_status;
+
+typedef enum { MOE_SOFTMAX = 0, MOE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Routing configuration ([ENT] "Concrete Implementation" router arguments;
+ * [GL] section 3 Gate arguments n_groups / topk_groups). */
+typedef struct {
+    int32_t T;            /* tokens */
+    int32_t d;            /* hidden size (gate GEMM contraction length) */
+    int32_t N;            /* routed experts */
+    int32_t K;            /* experts per token */
+    int32_t score_fn;     /* moe_score_fn */
+    int32_t n_groups;     /* expert groups (1 = no group limit); N % n_groups == 0 */
+    int32_t topk_groups;  /* groups kept per token */
+    int32_t group_topn;   /* group score = sum of this many largest keys (2) */
+    int32_t renorm;       /* 1: weights = s_k / sum of chosen s; 0: weights = s_k */
+    float route_scale;    /* weights are multiplied by this (2.5 for V3 routing) */
+    int32_t in_dtype;     /* moe_dtype of x and w_gate */
+} moe_route_cfg;
+
+/* Load statistics of one histogram, written to device memory.
+ * [MIN] "Run the example": total, max, mean, imbalance = max / mean (0 when
+ * mean is 0), capacity_fixed = max * n_slots.  [HD] "Deployment parameters
+ * and monitoring": std_over_mean (population std).  [ENT] "The Mathematics":
+ * entropy_load_bits = -sum p log2 p over p = count / total;
+ * "Concrete Implementation": entropy_score_bits = entropy of the batch-mean
+ * routing distribution (NaN when no scores were given);
+ * "Production Testing": capacity_125 = 1.25 * mean. */
+typedef struct {
+    int32_t status;       /* MOE_OK, or MOE_ERR_TIMEOUT if the offsets scan gave up */
+    int32_t n_slots;
+    int64_t total;
+    int64_t max_load;
+    double mean;
+    double imbalance;
+    double std_over_mean;
+    double entropy_load_bits;
+    double entropy_score_bits;
+    double capacity_fixed;
+    double capacity_125;
+} moe_stats;
+
+/* Bytes of workspace the calls below need for T tokens, K choices, N experts
+ * and n_slots histogram slots (n_slots >= N; N + replicas).  One workspace
+ * may serve every call on one stream; calls that overlap on the GPU need
+ * their own workspaces.  Contents need no initialisation. */
+size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
+
+/*
+ * moe_route -- gate GEMM, score nonlinearity, selection and combine weights.
+ *
+ * Gate ([ENT] "The Mathematics": h = x . W_g; "Concrete Implementation":
+ * nn.Linear(hidden, N, bias=False)):
+ *   h[t,e] = sum_j x[t,j] * w_gate[e,j] + logit_offset[e]
+ *   x [T,d], w_gate [N,d] in cfg->in_dtype (bf16: tcgen05 tensor-core GEMM
+ *   with fp32 accumulation, N % 16 == 0 and N <= 256; fp32: SIMT fp32 GEMM);
+ *   logit_offset [N] fp32 or NULL.
+ * Scores, fused into the GEMM epilogue, written to scores [T,N] fp32:
+ *   softmax over N ([ENT] softmax equation) or sigmoid ([HD] "Token routing").
+ *   If x == NULL the call skips the GEMM and reads `scores` as input instead.
+ * Selection ([HD] "Auxiliary-loss-free load balancing": the bias steers only
+ * the choice; [GL] sections 1 and 3: group-limited routing):
+ *   key = fp32(s + bias) (bias [N] fp32 or NULL); with n_groups > 1 the
+ *   topk_groups groups with the best fp32 sum of their group_topn largest
+ *   keys are kept and the rest excluded; the K best keys among the kept
+ *   experts are chosen.  Order: key descending, ties to the lower index.
+ *   topk_idx [T,K] int32 in that order.
+ * Weights ([ENT] "Concrete Implementation" renormalisation; [HD] weighted
+ * combine by affinity): from the UNBIASED scores,
+ *   topk_w[t,k] = fp32(fp32(s_k / fp32-sum-in-k-order) * route_scale)
+ *   (renorm = 1) or fp32(s_k * route_scale) (renorm = 0).
+ * ws: workspace of moe_workspace_bytes() bytes (error word of the GEMM).
+ */
+moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate,
+                     const float* logit_offset, const float* bias, float* scores,
+                     int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/*
+ * moe_load_stats -- load histogram, expert offsets, stable in-expert ranks
+ * and load statistics.
+ *
+ * slot(t,k) = topk_idx[t,k], or, when replica_slot [N] is given (a replica
+ * slot id in [N, n_slots) or -1 per expert), the replica slot for odd t and
+ * the original for even t ([HD] redundant experts for prefill; [GL] section
+ * 2).  slot_idx [T,K] receives slot(t,k) (may be NULL).
+ * counts [n_slots]: c_e = #{(t,k) : slot = e}  ([ENT] bincount).
+ * offsets [n_slots + 1]: exclusive prefix of counts, offsets[n_slots] = T*K.
+ * rank [T,K]: number of earlier flat assignments (t',k') < (t,k) with the
+ *   same slot -- the row's place inside its expert's segment.
+ * stats (device, may be NULL): see moe_stats.  scores [T,N] fp32 (may be
+ *   NULL) adds entropy_score_bits, with score_fn telling softmax rows
+ *   (used as they are) from sigmoid rows (normalised per token).
+ * Offsets come from a single-pass decoupled look-back scan over per-block
+ * counts; its waits are bounded (stats->status = MOE_ERR_TIMEOUT on expiry).
+ */
+moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
+                          const int32_t* replica_slot, int32_t n_slots, int32_t* slot_idx,
+                          int32_t* counts, int32_t* offsets, int32_t* rank,
+                          const float* scores, int32_t score_fn, moe_stats* stats, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_replica_plan -- replica slots for the n_replicas hottest experts.
+ * Experts ranked by (count desc, index asc); the j-th gets slot N + j, the
+ * rest -1.  counts [N] int32 (a histogram over the N experts), replica_slot
+ * [N] int32 out.  ([HD] "Auxiliary-loss-free load balancing": hot experts
+ * get copies in prefill; [GL] section 2: 32 redundant experts.)
+ * n_replicas in [0, N].
+ */
+moe_status moe_replica_plan(const int32_t* counts, int32_t N, int32_t n_replicas,
+                            int32_t* replica_slot, moe_stream_t stream);
+
+/*
+ * moe_bias_update -- per-expert routing bias step, in place on bias [N].
+ * ([HD] "Auxiliary-loss-free load balancing": lower the bias of overloaded
+ * experts, raise it for underloaded ones.)
+ *   mode 0: b_e = fp32(b_e - fp32(u * sign(c_e - total/N))), the sign taken
+ *           exactly on integers (c_e * N against total), sign(0) = 0.
+ *   mode 1: the proportional rule of [ENT] "Concrete Implementation" with
+ *           u as bias_decay: target = total / N, err = c_e - target,
+ *           b_e -= u * sign(err) * (|err| / target), every op fp32.
+ * counts [N] int32; total_assignments = T*K (> 0).
+ */
+moe_status moe_bias_update(const int32_t* counts, int32_t N, int64_t total_assignments,
+                           float u, int32_t mode, float* bias, moe_stream_t stream);
+
+/*
+ * moe_dispatch -- scatter token rows into the expert-contiguous buffer
+ * ([HD] "DeepEP": dispatch sends each token to its experts; FP8 dispatch).
+ *   pos[t,k] = offsets[slot_idx[t,k]] + rank[t,k]
+ *   rows[pos[t,k], :] = x[t, :]          (x_dtype, [T*K, d]; may be NULL)
+ *   row_src[pos[t,k]] = t               ([T*K] int32; may be NULL)
+ *   pos [T,K] int32 (may be NULL)
+ * FP8 copy (rows_fp8 [T*K, d] e4m3 bytes and scales [T*K, d/128] fp32, both
+ * NULL or both set; needs d % 128 == 0): per row and 128-channel block,
+ *   amax = max|v|, inv = amax > 0 ? fp32(448 / amax) : 0,
+ *   q = e4m3_rn_satfinite(fp32(v * inv)), scale = fp32(amax / 448).
+ * slot_idx, offsets, rank as produced by moe_load_stats.  d % 8 == 0
+ * (bf16) or d % 4 == 0 (fp32).
+ */
+moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, int32_t K,
+                        const int32_t* slot_idx, const int32_t* offsets, const int32_t* rank,
+                        void* rows, uint8_t* rows_fp8, float* scales, int32_t* pos,
+                        int32_t* row_src, moe_stream_t stream);
+
+/*
+ * moe_combine -- weighted gather-sum of expert outputs back to token order
+ * ([HD] "Token routing": outputs summed weighted by affinity; "DeepEP":
+ * combine, BF16).
+ *   out[t, :] = sum_{k=0..K-1} w[t,k] * y[pos[t,k], :]
+ * accumulated in fp32 in k order, rounded once to the output dtype.
+ * y [T*K, d] and out [T, d] in `dtype`; pos [T,K] int32, w [T,K] fp32.
+ */
+moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32_t K,
+                       const int32_t* pos, const float* w, void* out, moe_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the workspace's device error
+ * words: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait ran out since the last
+ * check.  (The only call that synchronises.) */
+moe_status moe_workspace_status(void* ws, moe_stream_t stream);
+
+/* Kernel launches issued by this library on the calling thread since the
+ * last reset (for launch accounting). */
+int64_t moe_launch_count(int32_t reset);
+
+const char* moe_status_str(moe_status s);
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_ROUTE_H_ */

@@ -1,0 +1,124 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry
+point the header declares, and rejects bad arguments on the host before any
+launch (no GPU needed: the rejected calls never reach CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_route.h")
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from expert_load_balancing_tcgen05_b200 import build
+    build.build()
+    from expert_load_balancing_tcgen05_b200 import moe as m
+    return m
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = _declared()
+    for n in ("moe_route", "moe_load_stats", "moe_bias_update", "moe_dispatch", "moe_combine"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(moe.EXPORTS) <= set(_declared())
+
+
+def test_version_and_status_strings(moe):
+    assert "sm_100a" in moe.moe_version()
+    assert moe._lib.moe_status_str(moe.MOE_ERR_TIMEOUT).decode() == "bounded device wait timed out"
+
+
+def test_workspace_bytes(moe):
+    a = moe.moe_workspace_bytes(16384, 8, 256)
+    b = moe.moe_workspace_bytes(131072, 8, 256, 288)
+    assert 0 < a < b < 4 << 20
+    assert moe.moe_workspace_bytes(100, 8, 256, 200) == 0   # n_slots < N
+    assert moe.moe_workspace_bytes(0, 8, 16) > 0
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def _cfg(moe, **kw):
+    c = dict(T=64, d=128, N=256, K=8, score_fn=1, n_groups=8, topk_groups=4, group_topn=2, renorm=1,
+             route_scale=2.5, in_dtype=1)
+    c.update(kw)
+    return moe.RouteCfg(**c)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=0), 1), (dict(K=300), 1), (dict(n_groups=3), 1), (dict(topk_groups=0), 1),
+    (dict(topk_groups=9), 1), (dict(group_topn=33), 1), (dict(score_fn=5), 1),
+    (dict(n_groups=8, topk_groups=1, K=40), 1), (dict(N=96, n_groups=1, K=8), 2),
+    (dict(N=256, n_groups=64, topk_groups=8), 1), (dict(N=24, n_groups=2, topk_groups=1, K=4), 2),
+])
+def test_route_rejects_bad_config(moe, kw, status):
+    cfg = _cfg(moe, **kw)
+    r = moe._lib.moe_route(ctypes.byref(cfg), None, None, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None)
+    assert r == status
+
+
+def test_route_rejects_null_outputs_and_workspace(moe):
+    cfg = _cfg(moe)
+    L = moe._lib
+    assert L.moe_route(None, None, None, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), None, None, None, None, MISALIGNED, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    # gate requested without weights / with a short workspace
+    assert L.moe_route(ctypes.byref(cfg), FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.moe_route(ctypes.byref(cfg), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, 16, None) == 1
+
+
+def test_load_stats_rejects_bad_arguments(moe):
+    L = moe._lib
+    ws = 1 << 24
+    assert L.moe_load_stats(FAKE, 64, 8, 256, None, 200, None, FAKE, FAKE, FAKE, None, 1, None, FAKE, ws, None) == 1
+    assert L.moe_load_stats(FAKE, 64, 8, 256, None, 288, None, FAKE, FAKE, FAKE, None, 1, None, FAKE, ws, None) == 1
+    assert L.moe_load_stats(FAKE, 64, 8, 256, None, 256, None, FAKE, FAKE, FAKE, None, 1, None, FAKE, 8, None) == 1
+    assert L.moe_load_stats(None, 64, 8, 256, None, 256, None, FAKE, FAKE, FAKE, None, 1, None, FAKE, ws, None) == 1
+    assert L.moe_load_stats(FAKE, 1 << 28, 16, 256, None, 256, None, FAKE, FAKE, FAKE, None, 1, None, FAKE, ws,
+                            None) == 1
+
+
+def test_dispatch_and_combine_reject_bad_arguments(moe):
+    L = moe._lib
+    # d not a multiple of 8 for bf16; FP8 without scales; FP8 with d % 128 != 0; misaligned rows
+    assert L.moe_dispatch(FAKE, 1, 10, 100, 8, FAKE, FAKE, FAKE, FAKE, None, None, None, None, None) == 1
+    assert L.moe_dispatch(FAKE, 1, 10, 256, 8, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None) == 1
+    assert L.moe_dispatch(FAKE, 1, 10, 136, 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == 1
+    assert L.moe_dispatch(FAKE, 1, 10, 256, 8, FAKE, FAKE, FAKE, MISALIGNED, None, None, None, None, None) == 1
+    assert L.moe_dispatch(FAKE, 7, 10, 256, 8, FAKE, FAKE, FAKE, FAKE, None, None, None, None, None) == 1
+    assert L.moe_combine(FAKE, 1, 10, 256, 33, FAKE, FAKE, FAKE, None) == 1
+    assert L.moe_combine(FAKE, 1, 10, 256, 8, FAKE, FAKE, MISALIGNED, None) == 1
+    assert L.moe_combine(None, 1, 10, 256, 8, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_bias_update_and_replica_plan_reject_bad_arguments(moe):
+    L = moe._lib
+    assert L.moe_bias_update(FAKE, 256, 0, 0.001, 0, FAKE, None) == 1
+    assert L.moe_bias_update(FAKE, 256, 100, 0.001, 2, FAKE, None) == 1
+    assert L.moe_bias_update(None, 256, 100, 0.001, 0, FAKE, None) == 1
+    assert L.moe_replica_plan(FAKE, 256, 257, FAKE, None) == 1
+    assert L.moe_replica_plan(FAKE, 256, -1, FAKE, None) == 1
+    assert L.moe_workspace_status(None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors(moe):
+    import torch
+    with pytest.raises(ValueError):
+        moe._ptr(torch.zeros(4))

@@ -1,0 +1,101 @@
+"""GPU parity of the gate GEMM + score nonlinearity (tcgen05 tensor-core
+kernel for bf16, CUDA-core kernel for fp32) against the fp64 oracle on the
+same inputs: scores within 1e-3 relative; the selection made from the GPU's
+own scores bit-exact against the oracle's selection on those scores; and
+against the oracle's own scores, differing only on near ties (gap < 1e-3)."""
+import numpy as np
+import pytest
+import torch
+
+from expert_load_balancing_tcgen05_b200 import workloads as W
+from gpu_util import gap_ok, lib, route_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+
+
+def _check_scores(s_gpu, s_ref):
+    err = np.abs(s_gpu.astype(np.float64) - s_ref.astype(np.float64))
+    bad = err > RTOL * np.abs(s_ref) + 1e-7
+    assert not bad.any(), (int(bad.sum()), float(err.max()))
+
+
+def _run_and_check(orc, wl, T, d, seed, check_gap=True):
+    wl = wl.with_(T=T, d=d)
+    inp = W.make_inputs(wl, seed=seed)
+    x, Wg, b, off = inp["x"], inp["W"], inp["bias"], inp["off"]
+    s_gpu, idx, w, ws = route_gpu(wl, x.cuda(), Wg.cuda(), off.cuda() if off is not None else None,
+                                  b.cuda() if b is not None else None)
+    assert lib().moe_workspace_status(ws) == 0
+    h = orc.logits(x.float().numpy(), Wg.float().numpy(), off.numpy() if off is not None else None)
+    s_ref = orc.scores(h, wl.fn)
+    sg = to_np(s_gpu)
+    _check_scores(sg, s_ref)
+    bn = b.numpy() if b is not None else None
+    # selection on the GPU's own scores: bit-exact
+    ri, rw = orc.select(sg, bn, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+    assert np.array_equal(to_np(idx), ri)
+    assert np.array_equal(to_np(w), rw)
+    if check_gap:
+        ri2, _ = orc.select(s_ref, bn, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+        diff, bad = gap_ok(s_ref, bn, to_np(idx), ri2, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn)
+        assert not bad, bad[:10]
+    return sg, s_ref
+
+
+TC_CASES = [
+    # workload, T, d
+    ("v3_router", 421, 7168),        # 4 tiles, ragged token tail, 112 k-steps
+    ("v3_router", 128, 1000),        # ragged k tail (1000 = 15*64 + 40)
+    ("v3_router", 1, 64),            # one token, one k-step
+    ("collapse", 300, 7168),         # celebrity logit offsets
+    ("prefill_replicas", 260, 7168),  # Zipf logit offsets
+    ("softmax_dispatch", 389, 4096),  # N=128 softmax
+]
+
+
+@pytest.mark.parametrize("name,T,d", TC_CASES)
+def test_gate_tc_against_oracle(orc, name, T, d):
+    _run_and_check(orc, W.WORKLOADS[name], T, d, seed=T + d)
+
+
+def test_gate_tc_n64_sigmoid(orc):
+    wl = W.Workload("n64", 0, 0, 0, 64, 6, fn=1, n_groups=4, topk_groups=2, scale=1.0, has_bias=True)
+    _run_and_check(orc, wl, 700, 512, seed=3)
+
+
+def test_gate_tc_many_tiles_per_cta(orc):
+    """More tiles than SMs: every CTA runs 2-3 tiles, so both TMEM
+    accumulators and every ring-slot phase are exercised."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    T = sms * 128 * 2 + 77
+    wl = W.WORKLOADS["softmax_dispatch"]
+    _run_and_check(orc, wl, T, 256, seed=11)
+
+
+def test_gate_simt_fp32_tiny_router(orc):
+    """The tiny softmax top-2 router of 8 experts, fp32, end to end."""
+    wl = W.WORKLOADS["tiny_softmax"]
+    _run_and_check(orc, wl, wl.T, wl.d, seed=wl.seed)
+
+
+def test_gate_simt_bf16_small_n(orc):
+    wl = W.Workload("n8bf16", 0, 0, 0, 8, 2, fn=0)
+    _run_and_check(orc, wl, 333, 256, seed=5)
+
+
+def test_zero_gate_gives_uniform_scores():
+    wl = W.WORKLOADS["v3_router"].with_(T=256, d=512)
+    x = torch.randn(256, 512, device="cuda").to(torch.bfloat16)
+    Wg = torch.zeros(256, 512, device="cuda", dtype=torch.bfloat16)
+    s, idx, _, _ = route_gpu(wl, x, Wg, None, None)
+    assert torch.all(s == 0.5)
+    # all-equal scores select the lowest experts (ties to the lower index)
+    assert torch.equal(idx.cpu(), torch.arange(8, dtype=torch.int32).expand(256, 8))
