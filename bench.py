@@ -1,0 +1,492 @@
+"""Benchmark of the MoE routing hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    (N > 1: launched by torch.distributed.run, one process per GPU)
+
+One step = one pass of the routing path over one batch of the throughput
+workload (T=16384 tokens, d=7168, N=256 experts, K=8, sigmoid scores, 8 groups
+keep 4, bias, weights x2.5):
+  moe_route       gate GEMM (tcgen05) + sigmoid + group-limited top-K + weights
+  moe_load_stats  histogram, look-back offsets, in-expert ranks, load stats
+  moe_bias_update sign-rule bias step
+  moe_dispatch    bf16 rows into the expert-contiguous buffer (+ positions)
+Combine is timed in its own loop (identity experts: it gathers the
+dispatched rows back) and reported under "stages".
+
+Metric: routed tokens/s = tokens of all ranks / max-over-ranks device time.
+Inputs are synthetic (seeded, drawn on the device) and larger than L2, so no
+flush is needed between steps.  Rank 0 prints one JSON line.
+
+--impl reference runs the CPU oracle (the plain fp64 restatement the tests
+use) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s (gate+topK+hist+dispatch) T=16K N=256 K=8; % roofline"
+UNIT = "tokens/s"
+WORKLOAD_NAME = "metric"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), \
+            "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: T={wl.T} d={wl.d} N={wl.N} K={wl.K} sigmoid, {wl.n_groups} groups keep "
+                        f"{wl.topk_groups}, group score top-{wl.group_topn} sum, bias U(-0.01,0.01), "
+                        f"weights x{wl.scale}, bf16 x~N(0,1) W~N(0,1/d)",
+            "T": wl.T, "d": wl.d, "N": wl.N, "K": wl.K, "global_batch": None,
+            "l2": "inputs larger than L2 (x 235 MB, dispatch buffer 1.88 GB per rank); no flush"}
+
+
+# --------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        return rows
+
+    @staticmethod
+    def summarise(rows):
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        loaded = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# --------------------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------------------
+class Pipeline:
+    """Device buffers and the sequence of library calls of one step."""
+
+    def __init__(self, wl, rank: int, device):
+        import torch
+        from expert_load_balancing_tcgen05_b200 import moe
+        from expert_load_balancing_tcgen05_b200 import workloads as W
+        self.moe, self.wl, self.dev = moe, wl, device
+        T, d, N, K = wl.T, wl.d, wl.N, wl.K
+        inp = W.make_inputs(wl, device=device, seed=wl.seed + 100 * rank)
+        self.x, self.W, self.bias0 = inp["x"], inp["W"], inp["bias"]
+        self.bias = self.bias0.clone()
+        self.off = inp["off"]
+        f32, i32 = torch.float32, torch.int32
+        self.scores = torch.empty(T, N, dtype=f32, device=device)
+        self.idx = torch.empty(T, K, dtype=i32, device=device)
+        self.w = torch.empty(T, K, dtype=f32, device=device)
+        self.slot = torch.empty(T, K, dtype=i32, device=device)
+        self.counts = torch.empty(N, dtype=i32, device=device)
+        self.offsets = torch.empty(N + 1, dtype=i32, device=device)
+        self.rank = torch.empty(T, K, dtype=i32, device=device)
+        self.pos = torch.empty(T, K, dtype=i32, device=device)
+        self.stats = moe.empty_stats(device)
+        self.ws = moe.workspace(T, K, N, N, device=device)
+        self.rows = torch.empty(T * K, d, dtype=torch.bfloat16, device=device)
+        self.out = torch.empty(T, d, dtype=torch.bfloat16, device=device)
+        self.cfg = moe.route_cfg(T, d, N, K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm,
+                                 wl.scale, moe.MOE_BF16)
+
+    def route(self, x=None):
+        self.moe.moe_route(self.cfg, self.x if x is None else x, self.W, self.off, self.bias, self.scores, self.idx,
+                           self.w, self.ws)
+
+    def load_stats(self):
+        wl = self.wl
+        self.moe.moe_load_stats(self.idx, wl.T, wl.K, wl.N, None, wl.N, self.slot, self.counts, self.offsets,
+                                self.rank, None, wl.fn, self.stats, self.ws)
+
+    def bias_update(self):
+        self.moe.moe_bias_update(self.counts, self.wl.N, self.wl.T * self.wl.K, 0.001, 0, self.bias)
+
+    def dispatch(self, x=None):
+        wl = self.wl
+        self.moe.moe_dispatch(self.x if x is None else x, wl.T, wl.d, wl.K, self.slot, self.offsets, self.rank,
+                              self.rows, None, None, self.pos, None)
+
+    def combine(self):
+        wl = self.wl
+        self.moe.moe_combine(self.rows, wl.T, wl.d, wl.K, self.pos, self.w, self.out)
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.route()
+        if ev is not None:
+            ev[1].record()
+        self.load_stats()
+        self.bias_update()
+        if ev is not None:
+            ev[2].record()
+        self.dispatch()
+        if ev is not None:
+            ev[3].record()
+
+
+def stage_bytes(wl):
+    """Algorithmic bytes / flops per launch (per batch of T tokens)."""
+    T, d, N, K = wl.T, wl.d, wl.N, wl.K
+    A = T * K
+    return {
+        "gate": {"bytes": T * d * 2 + N * d * 2 + T * N * 4, "flops": 2 * T * d * N},
+        "topk": {"bytes": T * N * 4 + N * 4 + A * 8},
+        "hist": {"bytes": A * 4 * 2 + A * 4 + (N + 1) * 4 * 2},   # idx read, slot+rank write, rank rw, offsets
+        "dispatch": {"bytes": T * d * 2 + A * d * 2 + A * 12},     # x once, K row copies, slot/rank in, pos out
+        "combine": {"bytes": A * d * 2 + A * 8 + T * d * 2},       # K rows in, pos/w in, token row out
+    }
+
+
+def pipeline_roofline_us(wl, hbm_gbs, tflops):
+    b = stage_bytes(wl)
+    t = 0.0
+    for k in ("gate", "topk", "hist", "dispatch"):
+        tb = b[k]["bytes"] / (hbm_gbs * 1e9)
+        tf = b[k].get("flops", 0) / (tflops * 1e12)
+        t += max(tb, tf)
+    return t * 1e6
+
+
+def _traffic_for(kernel_file: str, summary: str):
+    """dram bytes per launch from a committed ncu summary, if the kernel
+    source is unchanged since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "expert_load_balancing_tcgen05_b200", "csrc", kernel_file)
+    if not (os.path.exists(p) and os.path.exists(src)):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if j.get("source_sha256") != h:
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from expert_load_balancing_tcgen05_b200 import moe
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[WORKLOAD_NAME]
+    P = Pipeline(wl, rank, dev)
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up (also ramps clocks) and a correctness status check
+    for _ in range(max(args.warmup, 3)):
+        P.step()
+    torch.cuda.synchronize()
+    st = moe.moe_workspace_status(P.ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device-side status {st} after warm-up")
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    # soak ~0.3 s so the sampler sees the loaded clock before and during timing
+    t_end = time.time() + 0.3
+    while time.time() < t_end:
+        P.step()
+    torch.cuda.synchronize()
+
+    E = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    moe.moe_launch_count(reset=True)
+    barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(args.steps):
+        P.step(E[i])
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    launches = moe.moe_launch_count()
+    # keep the sampler running over a few more steps so short timed regions still get samples
+    t_end = time.time() + 0.2
+    while time.time() < t_end:
+        P.step()
+    torch.cuda.synchronize()
+    clocks = sampler.summarise(sampler.stop())
+
+    ms = start.elapsed_time(stop)
+    t_route = statistics.mean(E[i][0].elapsed_time(E[i][1]) for i in range(args.steps))
+    t_stats = statistics.mean(E[i][1].elapsed_time(E[i][2]) for i in range(args.steps))
+    t_disp = statistics.mean(E[i][2].elapsed_time(E[i][3]) for i in range(args.steps))
+
+    # combine: own loop (identity experts: gathers the dispatched rows back)
+    for _ in range(3):
+        P.combine()
+    cs, ce = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    cs.record()
+    for _ in range(args.steps):
+        P.combine()
+    ce.record()
+    torch.cuda.synchronize()
+    t_comb = cs.elapsed_time(ce) / args.steps
+
+    # max over ranks
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    tokens = wl.T * args.steps * world
+    value = tokens / (ms_max / 1e3)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # tokens, the routing path, D2H of the routing result (idx, weights,
+    # offsets, counts, stats); the dispatched rows stay on the device for the
+    # expert GEMMs.
+    x_host = P.x.cpu().pin_memory()
+    x_dev = torch.empty_like(P.x)
+    res = [P.idx, P.w, P.offsets, P.counts, P.stats]
+    res_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res]
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = sum(r.numel() * r.element_size() for r in res)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        P.route(x_dev); P.load_stats(); P.bias_update(); P.dispatch(x_dev)
+        for r, h in zip(res, res_host):
+            h.copy_(r, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record()
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        P.route(x_dev); P.load_stats(); P.bias_update(); P.dispatch(x_dev)
+        for r, h in zip(res, res_host):
+            h.copy_(r, non_blocking=True)
+    ee.record()
+    torch.cuda.synchronize()
+    te = torch.tensor([es.elapsed_time(ee)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = wl.T * e2e_steps * world / (float(te.item()) / 1e3)
+
+    b = stage_bytes(wl)
+    disp_bytes = b["dispatch"]["bytes"]
+    achieved = disp_bytes / (t_disp / 1e3) / 1e9
+    traffic = _traffic_for("dispatch_combine.cu", "dispatch_metric_dram.json")
+    roof_us = pipeline_roofline_us(wl, hbm, tf_burst)
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**workload_config(wl), "parallelism": f"dp{world} (independent token batches)"},
+            "roofline": {"bound": "hbm", "kernel": "dispatch_kernel", "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                         "bytes_per_launch": disp_bytes, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+            "pipeline_roofline": {"time_us": roof_us, "frac": roof_us / (ms_max / args.steps * 1e3),
+                                  "tokens_per_s_at_roofline": wl.T / (roof_us / 1e6),
+                                  "rule": "sum over gate/topK/hist/dispatch of max(flops/bf16 burst peak, "
+                                          "bytes/HBM peak)"},
+            "stages": {
+                "route_ms": t_route, "load_stats_and_bias_ms": t_stats, "dispatch_ms": t_disp,
+                "combine_ms": t_comb,
+                "gate_topk_gbs_equiv": (b["gate"]["bytes"] + b["topk"]["bytes"]) / (t_route / 1e3) / 1e9,
+                "gate_tflops_lower_bound": b["gate"]["flops"] / (t_route / 1e3) / 1e12,
+                "dispatch_gbs": achieved,
+                "combine_gbs": b["combine"]["bytes"] / (t_comb / 1e3) / 1e9,
+            },
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+    return out
+
+
+def cpu_baseline(seconds: float = 12.0):
+    """The oracle, as it stands, on the host cores: fp64 gate + scores +
+    selection + histogram/positions + dispatch rows for a sample of tokens of
+    the throughput workload; tokens/s scaled from the sample."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    wl = W.WORKLOADS[WORKLOAD_NAME]
+
+    def run(n):
+        sw = wl.with_(T=n)
+        inp = W.make_inputs(sw, seed=wl.seed)
+        x = inp["x"].float().numpy()
+        Wg = inp["W"].float().numpy()
+        b = inp["bias"].numpy()
+        x16 = inp["x"].view(torch.int16).numpy()
+        t0 = time.perf_counter()
+        h = oracle.logits(x, Wg)
+        s = oracle.scores(h, wl.fn)
+        idx, w = oracle.select(s, b, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+        counts, offsets, pos, rk, src = oracle.positions(idx, wl.N)
+        oracle.load_stats(counts)
+        oracle.bias_update(counts, n * wl.K, b, 0.001, 0)
+        oracle.dispatch_rows(x16, pos)
+        return time.perf_counter() - t0
+
+    probe = 64
+    tp = run(probe)
+    n = int(max(probe, min(wl.T, probe * seconds / max(tp, 1e-3))))
+    dt = run(n)
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of the {WORKLOAD_NAME} workload (T={wl.T} d={wl.d} N={wl.N} K={wl.K}): "
+                      f"fp64 gate, scores, grouped top-K, histogram/positions, stats, bias step, dispatch rows; "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: W warm-up + K timed steps, each a
+    bounded sample of the throughput workload."""
+    import oracle
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    import torch
+    wl = W.WORKLOADS[WORKLOAD_NAME]
+    n = int(os.environ.get("REF_SAMPLE_TOKENS", "1024"))
+    sw = wl.with_(T=n)
+    inp = W.make_inputs(sw, seed=wl.seed)
+    x = inp["x"].float().numpy()
+    Wg = inp["W"].float().numpy()
+    b = inp["bias"].numpy()
+    x16 = inp["x"].view(torch.int16).numpy()
+
+    def step():
+        h = oracle.logits(x, Wg)
+        s = oracle.scores(h, wl.fn)
+        idx, w = oracle.select(s, b, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+        counts, offsets, pos, rk, src = oracle.positions(idx, wl.N)
+        oracle.load_stats(counts)
+        oracle.bias_update(counts, n * wl.K, b, 0.001, 0)
+        oracle.dispatch_rows(x16, pos)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"{n} tokens per step of the {WORKLOAD_NAME} workload (T={wl.T} d={wl.d} N={wl.N} K={wl.K}), "
+              f"fp64 oracle on the host cores")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
