@@ -28,7 +28,7 @@ MOE_F32, MOE_BF16 = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
-           "moe_version")
+           "moe_version", "moe_load_stats_noalloc")
 
 
 class RouteCfg(ctypes.Structure):
@@ -115,6 +115,19 @@ def moe_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, o
     _check(_lib.moe_load_stats(_ptr(topk_idx), T, K, N, _ptr(replica_slot), n_slots, _ptr(slot_idx), _ptr(counts),
                                _ptr(offsets), _ptr(rank), _ptr(scores), score_fn, _ptr(stats), _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream)), "moe_load_stats")
+
+
+_lib.moe_load_stats_noalloc.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _P, _P, _I32, _P, _P]
+_lib.moe_load_stats_noalloc.restype = _I32
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_load_stats_noalloc(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets, rank, scores,
+                           score_fn, stats, stream=None):
+    """moe_load_stats with the library's fixed scratch array (for callers that cannot allocate)."""
+    _check(_lib.moe_load_stats_noalloc(_ptr(topk_idx), T, K, N, _ptr(replica_slot), n_slots, _ptr(slot_idx),
+                                       _ptr(counts), _ptr(offsets), _ptr(rank), _ptr(scores), score_fn,
+                                       _ptr(stats), _stream(stream)), "moe_load_stats_noalloc")
 
 
 def moe_replica_plan(counts, N, n_replicas, replica_slot, stream=None):

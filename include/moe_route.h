@@ -205,6 +205,37 @@ moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, in
 moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32_t K,
                        const int32_t* pos, const float* w, void* out, moe_stream_t stream);
 
+/*
+ * moe_load_stats_noalloc -- moe_load_stats without a caller workspace.  The
+ * pages have no counterpart: this is a library convenience.
+ *
+ * For callers that cannot allocate device memory where they call: a
+ * framework that owns the whole device memory pool, real-time or embedded
+ * code whose memory is fixed at start-up, host callbacks and plugins where a
+ * cudaMalloc would block or is not allowed.  Arguments and results are those
+ * of moe_load_stats; the scratch comes from a fixed device array inside this
+ * library of MOE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  The call allocates nothing.
+ *  - Returns MOE_ERR_UNSUPPORTED, enqueuing nothing, when the problem needs
+ *    more scratch than that (moe_workspace_bytes(T, K, N, n_slots) larger
+ *    than MOE_NOALLOC_SCRATCH_BYTES, 4 MiB; the largest routing workload
+ *    here, T = 131072 tokens, K = 8, 288 slots, needs about 1.1 MB).
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array, which keeps the last call's contents
+ *    (every call re-initialises what it needs).  Calls whose kernels overlap
+ *    on the GPU -- different streams, or threads, using the same device --
+ *    race on it and must be serialised by the caller.
+ * The load status of the call is in stats->status, as for moe_load_stats.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
+                                  const int32_t* replica_slot, int32_t n_slots, int32_t* slot_idx,
+                                  int32_t* counts, int32_t* offsets, int32_t* rank,
+                                  const float* scores, int32_t score_fn, moe_stats* stats,
+                                  moe_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the workspace's device error
  * words: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait ran out since the last
  * check.  (The only call that synchronises.) */
