@@ -1,14 +1,18 @@
 // C ABI of libmoeroute: argument validation on the host, then stream-ordered
 // launches.  No allocation, no synchronisation (except moe_workspace_status).
+#include <stddef.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 
 namespace moe {
 int route_epl(int N);
 bool gate_tc_supported(int N);
-cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, int T, int d, int N, int fn,
-                           float* scores, int32_t* err, cudaStream_t st);
+bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn);
+cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
+                           int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
+                           bool fused, float* scores, int32_t* idx, float* w, int32_t* err, cudaStream_t st);
 cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, int T, int d, int N,
                              int fn, float* scores, cudaStream_t st);
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K, int n_groups,
@@ -17,6 +21,7 @@ cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int
 cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const int32_t* replica_slot,
                               int n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets, int32_t* rank,
                               const float* scores, int score_fn, moe_stats* stats, void* ws, cudaStream_t st);
+cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t st);
 cudaError_t launch_replica_plan(const int32_t* counts, int N, int R, int32_t* replica_slot, cudaStream_t st);
 cudaError_t launch_bias_update(const int32_t* counts, int N, int64_t total, float u, int mode, float* bias,
                                cudaStream_t st);
@@ -47,6 +52,18 @@ int sm_count() {
 using namespace moe;
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Whether the GEMM epilogue selects (instead of a separate selection kernel).
+// The epilogue's selection is serial per token row; it pays off only when it
+// overlaps the next tile's main loop, i.e. when every CTA runs several tiles.
+// MOE_FUSED_SELECT=0/1 forces either path (tuning and tests).
+static bool use_fused_select(int T) {
+    const char* e = getenv("MOE_FUSED_SELECT");
+    if (e != nullptr && e[0] == '0') return false;
+    if (e != nullptr && e[0] == '1') return true;
+    const int tiles = (T + 127) / 128;
+    return tiles >= 3 * moe_host::sm_count();
+}
 static inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 static moe_status check_route_cfg(const moe_route_cfg* c) {
@@ -84,8 +101,13 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
     moe_status s = check_route_cfg(cfg);
     if (s != MOE_OK) return s;
     const moe_route_cfg& c = *cfg;
-    if (scores == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID;
-    if (!aligned16(scores)) return MOE_ERR_INVALID;
+    if (topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID;
+    if (scores != nullptr && !aligned16(scores)) return MOE_ERR_INVALID;
+    const int eff_topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
+    const bool tensor_core = x != nullptr && c.in_dtype == MOE_BF16 && gate_tc_supported(c.N);
+    const bool fused = tensor_core && gate_tc_can_fuse(c.N, c.K, c.score_fn, c.n_groups, c.group_topn) &&
+                       (scores == nullptr || use_fused_select(c.T));
+    if (scores == nullptr && !fused) return MOE_ERR_INVALID;  // the scores carry the selection's input
     if (c.T == 0) return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (x != nullptr) {
@@ -95,17 +117,18 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
         if (c.in_dtype != MOE_F32 && c.in_dtype != MOE_BF16) return MOE_ERR_INVALID;
         WsHeader* hdr = reinterpret_cast<WsHeader*>(static_cast<char*>(ws) + ws_layout(c.T, c.K, c.N, c.N).header);
         cudaError_t e;
-        if (c.in_dtype == MOE_BF16 && gate_tc_supported(c.N)) {
+        if (tensor_core) {
             if (c.d % 8 != 0 || !aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID;
-            e = cudaMemsetAsync(&hdr->gate_err, 0, sizeof(int32_t), st);
+            e = launch_gate_tc(x, w_gate, logit_offset, bias, c.T, c.d, c.N, c.K, c.score_fn, c.n_groups,
+                               eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, fused, scores,
+                               topk_idx, topk_w, &hdr->gate_err, st);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
-            e = launch_gate_tc(x, w_gate, logit_offset, c.T, c.d, c.N, c.score_fn, scores, &hdr->gate_err, st);
+            if (fused) return MOE_OK;
         } else {
             e = launch_gate_simt(x, w_gate, c.in_dtype, logit_offset, c.T, c.d, c.N, c.score_fn, scores, st);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    const int eff_topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
     return cuda_status(launch_route_topk(scores, bias, c.T, c.N, c.K, c.n_groups, eff_topk_groups,
                                          c.group_topn, c.renorm ? 1 : 0, c.route_scale, topk_idx, topk_w, st));
 }
@@ -176,18 +199,37 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
 moe_status moe_workspace_status(void* ws, moe_stream_t stream) {
     if (ws == nullptr) return MOE_ERR_INVALID;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    WsHeader h;
-    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    struct {
+        WsHeader h;
+        ScanCtl c;
+    } w;
+    static_assert(sizeof(w) == sizeof(WsHeader) + sizeof(ScanCtl), "header and control are adjacent");
+    if (cudaMemcpyAsync(&w, ws, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    const int32_t scan = w.c.sticky | w.c.err;
     moe_status r = MOE_OK;
-    if ((h.gate_err & 1) || (h.scan_err & 1)) r = MOE_ERR_TIMEOUT;
-    else if (h.scan_err & 2) r = MOE_ERR_INVALID;
-    if (h.gate_err || h.scan_err) {
-        int32_t z[2] = {0, 0};
-        if (cudaMemcpyAsync(ws, z, sizeof(z), cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((w.h.gate_err & 1) || (scan & 1)) r = MOE_ERR_TIMEOUT;
+    else if (scan & 2) r = MOE_ERR_INVALID;
+    if (w.h.gate_err || w.c.sticky) {
+        const int32_t z = 0;
+        char* base = static_cast<char*>(ws);
+        if (cudaMemcpyAsync(base + offsetof(WsHeader, gate_err), &z, sizeof(z), cudaMemcpyHostToDevice, st) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(base + sizeof(WsHeader) + offsetof(ScanCtl, sticky), &z, sizeof(z),
+                            cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
     }
     return r;
+}
+
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (ws == nullptr || ws_bytes < moe_workspace_bytes(2 * LS_BLOCK, 1, 8, 8)) return MOE_ERR_INVALID;
+    int32_t err = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (run_lookback_timeout_probe(ws, &err, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    return (err & 1) ? MOE_ERR_TIMEOUT : MOE_OK;
 }
 
 int64_t moe_launch_count(int32_t reset) {

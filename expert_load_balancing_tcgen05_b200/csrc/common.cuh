@@ -15,47 +15,69 @@ namespace moe {
 constexpr unsigned FULL = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
-// Workspace layout (all regions 256-byte aligned).  The header holds the
-// error words and the scan's tile ticket; the rest is per-call scratch.
+// Workspace layout (regions 256-byte aligned):
+//   header   256 B   gate error word (moe_route)
+//   ctl       64 B   per-call control of the load-statistics pass: tile
+//                    ticket, finished-block counter, error bits
+//   flags   4*nblk   look-back status per block: bit 31 | call epoch << 2 | state
+//                    (state 1 aggregate, 2 prefix); a word without this
+//                    call's tag -- zero, an older call's flag, or a count of
+//                    another layout (counts never have bit 31) -- means "none"
+//   agg     nblk x n_slots int32   per-block slot counts
+//   pre     nblk x n_slots int32   per-block inclusive prefix over blocks
+//   hs      HS_BLOCKS x N double   score-entropy partial column sums
+// The workspace is zero-filled once by its owner before first use.  Each
+// load-statistics call then leaves ctl ready for the next call (its last
+// block resets the ticket and finished counter and advances the epoch after
+// every other block is done); flags need no reset because they carry the
+// epoch; the error words are sticky until moe_workspace_status reads them.
 // ---------------------------------------------------------------------------
 struct WsHeader {
-    int32_t gate_err;       // set by the gate GEMM when a barrier wait runs out
-    int32_t scan_err;       // set by the offsets scan (look-back) or a bad id
-    uint32_t scan_ticket;   // dynamic tile counter of the look-back scan
-    int32_t pad[61];
+    int32_t gate_err;       // bit 0: a barrier wait of the gate GEMM ran out
+    int32_t pad[63];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
-constexpr int HIST_THREADS = 256;              // 8 warps
-constexpr int HIST_WARPS = HIST_THREADS / 32;
-constexpr int HIST_ITEMS_PER_WARP = 512;       // 16 chunks of 32 assignments
-constexpr int HIST_BLOCK = HIST_WARPS * HIST_ITEMS_PER_WARP;  // 4096 assignments per block
+struct ScanCtl {
+    uint32_t ticket;        // next block index to hand out
+    uint32_t done;          // blocks finished
+    int32_t err;            // this call: bit 0 look-back wait ran out; bit 1 expert id out of range
+    int32_t sticky;         // all calls since the last moe_workspace_status
+    uint32_t epoch;         // calls completed; tags this call's look-back flags
+    int32_t pad[11];
+};
+static_assert(sizeof(ScanCtl) == 64, "control block is 64 bytes");
+
+constexpr int LS_THREADS = 256;                // 8 warps
+constexpr int LS_WARPS = LS_THREADS / 32;
+constexpr int LS_CHUNKS = 8;                   // 32-assignment chunks per warp
+constexpr int LS_BLOCK = LS_WARPS * LS_CHUNKS * 32;  // 2048 assignments per block
 constexpr int MAX_SLOTS = 2048;                // smem: 8 warps x 2048 x 4 B = 64 KB
-constexpr int SCAN_THREADS = 256;
-constexpr int SCAN_ITEMS = 8;
-constexpr int SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;  // 2048 values per look-back tile
+constexpr int LS_SLOTS_PER_THREAD = MAX_SLOTS / LS_THREADS;
 constexpr int HS_BLOCKS = 256;                 // blocks of the score-entropy pass
 constexpr int MAX_N = 1024;                    // experts supported by selection / stats
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t header = 0, blk_counts = 0, blk_base = 0, scan_status = 0, hs_partial = 0, total = 0;
-    int64_t nblk = 0, L = 0, n_tiles = 0;
+    size_t header = 0, ctl = 0, flags = 0, agg = 0, pre = 0, hs_partial = 0, total = 0, ctl_bytes = 0;
+    int64_t nblk = 0;
 };
 
 inline WsLayout ws_layout(int64_t T, int32_t K, int32_t N, int32_t n_slots) {
     WsLayout w;
-    int64_t A = T * (int64_t)K;
-    w.nblk = (A + HIST_BLOCK - 1) / HIST_BLOCK;
+    const int64_t A = T * (int64_t)K;
+    w.nblk = (A + LS_BLOCK - 1) / LS_BLOCK;
     if (w.nblk < 1) w.nblk = 1;
-    w.L = w.nblk * (int64_t)n_slots;
-    w.n_tiles = (w.L + SCAN_TILE - 1) / SCAN_TILE;
+    const size_t cells = (size_t)w.nblk * (size_t)n_slots;
     size_t off = 0;
     w.header = off;      off += align256(sizeof(WsHeader));
-    w.blk_counts = off;  off += align256(sizeof(int32_t) * (size_t)w.L);
-    w.blk_base = off;    off += align256(sizeof(int32_t) * (size_t)w.L);
-    w.scan_status = off; off += align256(sizeof(uint64_t) * (size_t)w.n_tiles);
+    w.ctl = off;
+    w.flags = off + sizeof(ScanCtl);
+    w.ctl_bytes = sizeof(ScanCtl) + sizeof(uint32_t) * (size_t)w.nblk;
+    off += align256(w.ctl_bytes);
+    w.agg = off;         off += align256(sizeof(int32_t) * cells);
+    w.pre = off;         off += align256(sizeof(int32_t) * cells);
     w.hs_partial = off;  off += align256(sizeof(double) * (size_t)HS_BLOCKS * (size_t)(N > 0 ? N : 1));
     w.total = off;
     return w;
@@ -85,6 +107,16 @@ __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
 
 __device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {

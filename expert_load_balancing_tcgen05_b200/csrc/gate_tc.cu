@@ -25,15 +25,19 @@
 // the workspace, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "common.cuh"
+#include "select.cuh"
 
 namespace moe {
 namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;             // two per TMEM lane quarter, each owning half the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -147,16 +151,168 @@ struct Cfg {
     static constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;  // 128, 256 or 512: powers of two
-    static constexpr size_t SMEM_BYTES =
-        1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16 + 4 * BN;
+    // epilogue exchange (per token row): 2 x 2 reduction floats, up to 8 group
+    // scores, one 8-entry candidate list (key, score, index)
+    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8) * 4 + 2 * EPI_WARPS * 4;
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
+                                         8 * (2 * STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
+
+// Epilogue parameters.  `fused` = select in the epilogue (write topk_idx /
+// topk_w directly); otherwise only the scores are written.
+struct Epi {
+    const float* off;   // [N] logit offsets or null
+    const float* bias;  // [N] selection bias or null
+    float* scores;      // [T, N] or null (fused only)
+    int32_t* idx;       // [T, K]
+    float* w;           // [T, K]
+    int T, fn, K, n_groups, topk_groups, group_topn, renorm, fused;
+    float scale;
+};
+
+__device__ __forceinline__ void store32(float* dst, const float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+}
+
+// Named barrier over the epilogue warps only.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory"); }
+
+// Shared-memory exchange between the two warps that own one token row.
+struct Xch {
+    float* red;   // [2][2][BM]: per half, per round (max, then sum)
+    float* gs;    // [BM][8]: group scores
+    float* lk;    // [BM][8]: the second half's candidate list
+    float* ls;    // [BM][8]
+    int* li;      // [BM][8]
+    int* agree;   // [2][EPI_WARPS]: per tile parity, each warp's wait verdict
+};
+
+// One token row (this thread's TMEM lane) of one finished tile.  The two
+// warps of a lane quarter split the columns: half h owns chunks
+// [h*NC/2, (h+1)*NC/2) of 32 columns.  Softmax exchanges the row max and sum;
+// grouped selection exchanges group scores; half 1 hands its top-8 to half 0,
+// which merges and writes the row's choice.  Every epilogue thread executes
+// the same sequence of epi_sync() calls.
+template <int BN>
+__device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int row, int h, int64_t grow,
+                                             const float* off_s, const float* bias_s, const Xch& x) {
+    constexpr int NC = BN / 32, NCH = NC / 2;
+    const int c_lo = h * NCH;
+    const bool live = grow < p.T;
+    float* srow = (p.scores != nullptr && live) ? p.scores + grow * BN : nullptr;
+    float v[32];
+    Top8 top;
+    top.init();
+    if (p.fn == MOE_SIGMOID) {
+        if (p.fused && p.n_groups > 1) {
+            // one expert group per 32-column chunk: group score = sum of its top-n keys
+#pragma unroll
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int c = c_lo + cc;
+                tmem_ld32(taddr + 32 * c, v);
+                float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
+                    const float key = __fadd_rn(v[i], bias_s[32 * c + i]);
+                    if (key > t1) { t2 = t1; t1 = key; } else if (key > t2) { t2 = key; }
+                }
+                x.gs[row * 8 + c] = p.group_topn == 1 ? t1 : __fadd_rn(t1, t2);
+                if (srow) store32(srow + 32 * c, v);
+            }
+            epi_sync();
+            float gs[NC];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) gs[c] = x.gs[row * 8 + c];
+            unsigned keep = 0;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                int rank = 0;
+#pragma unroll
+                for (int c2 = 0; c2 < NC; ++c2) rank += (c2 != c && beats(gs[c2], c2, gs[c], c)) ? 1 : 0;
+                if (rank < p.topk_groups) keep |= 1u << c;
+            }
+#pragma unroll 1
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int c = c_lo + cc;
+                tmem_ld32(taddr + 32 * c, v);  // warp-collective: every lane loads every chunk
+                if ((keep >> c) & 1u) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float sv = sigmoid_f(v[i] + off_s[32 * c + i]);
+                        top.offer(__fadd_rn(sv, bias_s[32 * c + i]), 32 * c + i, sv);
+                    }
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int c = c_lo + cc;
+                tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
+                    if (p.fused) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
+                }
+                if (srow) store32(srow + 32 * c, v);
+            }
+        }
+    } else {
+        // softmax over the whole row: exchange the halves' max, then their sums
+        float m = -INFINITY;
+#pragma unroll 1
+        for (int cc = 0; cc < NCH; ++cc) {
+            const int c = c_lo + cc;
+            tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i] + off_s[32 * c + i]);
+        }
+        x.red[(h * 2 + 0) * BM + row] = m;
+        epi_sync();
+        m = fmaxf(x.red[0 * BM + row], x.red[2 * BM + row]);
+        float sum = 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < NCH; ++cc) {
+            const int c = c_lo + cc;
+            tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum += expf(v[i] + off_s[32 * c + i] - m);
+        }
+        x.red[(h * 2 + 1) * BM + row] = sum;
+        epi_sync();
+        const float inv = 1.f / (x.red[1 * BM + row] + x.red[3 * BM + row]);
+#pragma unroll 1
+        for (int cc = 0; cc < NCH; ++cc) {
+            const int c = c_lo + cc;
+            tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
+                if (p.fused) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
+            }
+            if (srow) store32(srow + 32 * c, v);
+        }
+    }
+    if (!p.fused) return;
+    // half 1 hands its list to half 0; its indices are all above half 0's,
+    // so offering them in list order keeps (key desc, index asc)
+    if (h == 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { x.lk[row * 8 + j] = top.k[j]; x.ls[row * 8 + j] = top.s[j]; x.li[row * 8 + j] = top.i[j]; }
+    }
+    epi_sync();
+    if (h == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) top.offer(x.lk[row * 8 + j], x.li[row * 8 + j], x.ls[row * 8 + j]);
+        if (live) top.write(p.K, p.renorm, p.scale, p.idx + grow * p.K, p.w + grow * p.K);
+    }
+}
 
 template <int BN>
 __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                             const __grid_constant__ CUtensorMap tmB, int T,
-                                                             int d, int fn, const float* __restrict__ off,
-                                                             float* __restrict__ scores, int32_t* err,
-                                                             int num_tiles) {
+                                                             const __grid_constant__ CUtensorMap tmB, int d,
+                                                             const Epi p, int32_t* err, int num_tiles) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -167,6 +323,14 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
+    float* bias_s = off_s + BN;
+    Xch xch;
+    xch.red = bias_s + BN;
+    xch.gs = xch.red + 4 * BM;
+    xch.lk = xch.gs + 8 * BM;
+    xch.ls = xch.lk + 8 * BM;
+    xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
+    xch.agree = xch.li + 8 * BM;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
@@ -176,7 +340,7 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(tfull0 + 8 * a, 1); mbar_init(tempty0 + 8 * a, 4); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull0 + 8 * a, 1); mbar_init(tempty0 + 8 * a, EPI_WARPS); }
         mbar_init(done_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -186,7 +350,10 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < BN; i += blockDim.x) off_s[i] = off != nullptr ? off[i] : 0.f;
+    for (int i = threadIdx.x; i < BN; i += blockDim.x) {
+        off_s[i] = p.off != nullptr ? p.off[i] : 0.f;
+        bias_s[i] = p.bias != nullptr ? p.bias[i] : 0.f;
+    }
     fence_before();
     __syncthreads();
     fence_after();
@@ -244,61 +411,25 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int h = (warp - 2) >> 2;       // which half of the columns
         const int row = q * 32 + lane;
         uint32_t local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const uint32_t a = local & 1, aph = (local >> 1) & 1;
-            // one lane waits, the warp follows its verdict together (tcgen05.ld is warp-collective)
+            // one lane per warp waits; the epilogue warps then agree on one verdict
+            // (tcgen05.ld is warp-collective and the halves meet at named barriers,
+            // so either every epilogue warp processes the tile or none does)
+            const int ew = warp - 2;
+            if (lane == 0) xch.agree[a * EPI_WARPS + ew] = mbar_wait(tfull0 + 8 * a, aph, err) ? 1 : 0;
+            epi_sync();
             int ok = 1;
-            if (lane == 0) ok = mbar_wait(tfull0 + 8 * a, aph, err) ? 1 : 0;
-            ok = __shfl_sync(FULL, ok, 0);
+#pragma unroll
+            for (int w = 0; w < EPI_WARPS; ++w) ok &= xch.agree[a * EPI_WARPS + w];
             if (!ok) break;
             fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + a * BN;
             const int64_t grow = (int64_t)tile * BM + row;
-            float* out = scores + grow * BN;
-            const bool live = grow < T;
-            float v[32];
-            if (fn == MOE_SIGMOID) {
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    tmem_ld32(taddr + c0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 1.f / (1.f + expf(-(v[i] + off_s[c0 + i])));
-                    if (live) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(out + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    }
-                }
-            } else {
-                float m = -INFINITY;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    tmem_ld32(taddr + c0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i] + off_s[c0 + i]);
-                }
-                float sum = 0.f;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    tmem_ld32(taddr + c0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) sum += expf(v[i] + off_s[c0 + i] - m);
-                }
-                const float inv = 1.f / sum;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    tmem_ld32(taddr + c0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = expf(v[i] + off_s[c0 + i] - m) * inv;
-                    if (live) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(out + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    }
-                }
-            }
+            epilogue_row<BN>(p, taddr, row, h, grow, off_s, bias_s, xch);
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty0 + 8 * a);
@@ -311,6 +442,229 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     if (warp == 1) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+
+// ===========================================================================
+// Two-SM variant (N = 256): a cluster of two CTAs computes a 256-token tile
+// with tcgen05.mma.cta_group::2 (M = 256 across the pair, N = 256).  Each CTA
+// loads its own 128 token rows of x and its own half (128 experts) of W per
+// k-step, so a stage is 32 KB per SM instead of 48 KB: half the W traffic
+// from L2 and a third less shared-memory traffic per MMA, with six stages in
+// flight.  The leader CTA (rank 0) owns the full barriers (both CTAs' TMA
+// loads complete on them), issues the MMAs, and multicasts its commits to
+// both CTAs' barriers; each CTA's TMEM receives its own 128 rows x 256
+// columns and each CTA runs the same epilogue on them.
+// ===========================================================================
+constexpr int PAIR_STAGES = 6;
+constexpr uint32_t PAIR_STAGE_BYTES = 2u * BM * BK * 2;  // A rows + B half, per CTA
+struct PairCfg {
+    static constexpr int BN = 256;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr size_t XCH_BYTES = Cfg<256>::XCH_BYTES;
+    static constexpr size_t SMEM_BYTES = 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES +
+                                         8 * (2 * PAIR_STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// address of the same shared-memory object in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// leader CTA's barrier (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(id), "r"(acc)
+        : "memory");
+}
+
+// commit this thread's MMAs to the barrier at `bar` in both CTAs of the pair
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_pair_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// bf16 x bf16 -> fp32, K-major, M = 256 (pair), N = 256
+__device__ __forceinline__ constexpr uint32_t idesc_pair() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    gate_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int d,
+                        const Epi p, int32_t* err, int num_pairs) {
+    constexpr int BN = 256, STAGES = PAIR_STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;                                      // [STAGES][128 x 64] bf16, 128B swizzle
+    uint8_t* sB = smem + (size_t)STAGES * (BM * BK * 2);     // [STAGES][128 x 64] bf16 (this CTA's experts)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * PAIR_STAGE_BYTES);
+    // bars: full[STAGES] (leader), empty[STAGES], tfull[2], tempty[2] (leader), done (leader)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
+    float* bias_s = off_s + BN;
+    Xch xch;
+    xch.red = bias_s + BN;
+    xch.gs = xch.red + 4 * BM;
+    xch.lk = xch.gs + 8 * BM;
+    xch.ls = xch.lk + 8 * BM;
+    xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
+    xch.agree = xch.li + 8 * BM;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+    const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
+    const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+    const int num_kb = (d + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull0 + 8 * a, 1); mbar_init(tempty0 + 8 * a, 2 * EPI_WARPS); }
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(PairCfg::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < BN; i += blockDim.x) {
+        off_s[i] = p.off != nullptr ? p.off[i] : 0.f;
+        bias_s[i] = p.bias != nullptr ? p.bias[i] : 0.f;
+    }
+    fence_before();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+    fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tp = cluster; tp < num_pairs && ok; tp += nclusters) {
+                const int m0 = tp * 2 * BM + (int)rank * BM;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
+                    const uint32_t fb = map_to(full0 + 8 * s, 0);
+                    if (leader) mbar_expect_tx(full0 + 8 * s, 2 * PAIR_STAGE_BYTES);
+                    tma_load_2d_pair(smem_u32(sA + (size_t)s * (BM * BK * 2)), &tmA, kb * BK, m0, fb);
+                    tma_load_2d_pair(smem_u32(sB + (size_t)s * (BM * BK * 2)), &tmB, kb * BK, (int)rank * BM, fb);
+                }
+            }
+            // drain: this CTA's last loads into each slot have landed (the leader sees all of them)
+            if (leader) {
+                const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+                for (uint32_t j = first; j < it; ++j) {
+                    const uint32_t s = j % STAGES, ph = (j / STAGES) & 1;
+                    if (!mbar_wait(full0 + 8 * s, ph, err, /*watch=*/false)) break;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            uint32_t it = 0, local = 0;
+            bool ok = true;
+            for (int tp = cluster; tp < num_pairs && ok; tp += nclusters, ++local) {
+                const uint32_t a = local & 1, aph = (local >> 1) & 1;
+                if (!mbar_wait(tempty0 + 8 * a, aph ^ 1, err)) { ok = false; break; }
+                fence_after();
+                const uint32_t d_tmem = tmem_base + a * BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!mbar_wait(full0 + 8 * s, ph, err)) { ok = false; break; }
+                    fence_after();
+                    const uint32_t a_addr = smem_u32(sA + (size_t)s * (BM * BK * 2));
+                    const uint32_t b_addr = smem_u32(sB + (size_t)s * (BM * BK * 2));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16_pair(d_tmem, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc_pair(),
+                                      (kb > 0 || k > 0) ? 1u : 0u);
+                    mma_commit_pair(empty0 + 8 * s);
+                }
+                if (ok) mma_commit_pair(tfull0 + 8 * a);
+            }
+            mma_commit_pair_local(done_bar);
+            mbar_wait(done_bar, 0, err, /*watch=*/false);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
+        const int row = q * 32 + lane;
+        const uint32_t tempty_leader0 = map_to(tempty0, 0);
+        uint32_t local = 0;
+        for (int tp = cluster; tp < num_pairs; tp += nclusters, ++local) {
+            const uint32_t a = local & 1, aph = (local >> 1) & 1;
+            const int ew = warp - 2;
+            if (lane == 0) xch.agree[a * EPI_WARPS + ew] = mbar_wait(tfull0 + 8 * a, aph, err) ? 1 : 0;
+            epi_sync();
+            int ok = 1;
+#pragma unroll
+            for (int w = 0; w < EPI_WARPS; ++w) ok &= xch.agree[a * EPI_WARPS + w];
+            if (!ok) break;
+            fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + a * BN;
+            const int64_t grow = (int64_t)tp * 2 * BM + (int64_t)rank * BM + row;
+            epilogue_row<BN>(p, taddr, row, h, grow, off_s, bias_s, xch);
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * a);
+        }
+    }
+
+    // both CTAs finished with TMEM and the leader's MMAs are drained before
+    // either CTA frees its half of the accumulators
+    fence_before();
+    __syncthreads();
+    cluster_sync();
+    fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(PairCfg::TMEM_COLS)
                      : "memory");
     }
 }
@@ -352,9 +706,33 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t col
 
 bool gate_tc_supported(int N) { return N == 64 || N == 128 || N == 256; }
 
+// The epilogue can select when the groups are whole 32-column chunks (or
+// there is one group) and K fits its 8-entry list.
+bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn) {
+    if (K > 8) return false;
+    if (n_groups == 1) return true;
+    return fn == MOE_SIGMOID && N / n_groups == 32 && group_topn >= 1 && group_topn <= 2;
+}
+
+static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const tc::Epi& p, int32_t* err,
+                               cudaStream_t st) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, 256, d, tc::BM)) return cudaErrorInvalidValue;
+    const size_t smem = tc::PairCfg::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(tc::gate_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int num_pairs = (T + 2 * tc::BM - 1) / (2 * tc::BM);
+    int clusters = moe_host::sm_count() / 2;
+    if (clusters > num_pairs) clusters = num_pairs;
+    if (clusters < 1) clusters = 1;
+    tc::gate_tc_pair_kernel<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);
+    moe_host::note_launch();
+    return cudaGetLastError();
+}
+
 template <int BN>
-static cudaError_t launch_bn(const void* x, const void* W, const float* off, int T, int d, int fn, float* scores,
-                             int32_t* err, cudaStream_t st) {
+static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const tc::Epi& p, int32_t* err,
+                             cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, BN, d, BN)) return cudaErrorInvalidValue;
     const size_t smem = tc::Cfg<BN>::SMEM_BYTES;
@@ -364,17 +742,26 @@ static cudaError_t launch_bn(const void* x, const void* W, const float* off, int
     int grid = moe_host::sm_count();
     if (grid > num_tiles) grid = num_tiles;
     if (grid < 1) grid = 1;
-    tc::gate_tc_kernel<BN><<<grid, tc::THREADS, smem, st>>>(ma, mb, T, d, fn, off, scores, err, num_tiles);
+    tc::gate_tc_kernel<BN><<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles);
     moe_host::note_launch();
     return cudaGetLastError();
 }
 
-cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, int T, int d, int N, int fn,
-                           float* scores, int32_t* err, cudaStream_t st) {
+cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
+                           int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
+                           bool fused, float* scores, int32_t* idx, float* w, int32_t* err, cudaStream_t st) {
+    tc::Epi p;
+    p.off = off; p.bias = bias; p.scores = scores; p.idx = idx; p.w = w;
+    p.T = T; p.fn = fn; p.K = K; p.n_groups = n_groups; p.topk_groups = topk_groups; p.group_topn = group_topn;
+    p.renorm = renorm; p.fused = fused ? 1 : 0; p.scale = scale;
     switch (N) {
-        case 64: return launch_bn<64>(x, W, off, T, d, fn, scores, err, st);
-        case 128: return launch_bn<128>(x, W, off, T, d, fn, scores, err, st);
-        case 256: return launch_bn<256>(x, W, off, T, d, fn, scores, err, st);
+        case 64: return launch_bn<64>(x, W, T, d, p, err, st);
+        case 128: return launch_bn<128>(x, W, T, d, p, err, st);
+        case 256: {
+            const char* e = getenv("MOE_GATE_PAIR");
+            const bool pair = e == nullptr || e[0] != '0';
+            return pair ? launch_pair(x, W, T, d, p, err, st) : launch_bn<256>(x, W, T, d, p, err, st);
+        }
         default: return cudaErrorInvalidValue;
     }
 }

@@ -10,102 +10,19 @@
 // layout that dispatch and combine use ("DeepSeek V4 MoE load balancing",
 // DeepEP section).
 //
-// Pipeline (one stream, no host synchronisation):
-//   hist_rank     per 4096-assignment block: slot remap, warp-private
-//                 shared-memory histograms, stable in-block rank via
-//                 __match_any_sync; writes per-block counts expert-major.
-//   scan          single-pass decoupled look-back exclusive scan over the
-//                 expert-major per-block counts -> every (expert, block) base.
-//   finalize      in-expert rank = base - offset + in-block rank; offsets and
-//                 counts.
-//   score_entropy optional: per-block column sums of normalised scores.
-//   stats         one block: moments, entropy, capacities, status.
+// One stream, no host synchronisation: the optional score-entropy column
+// sums, then one single-pass kernel (histogram, look-back, ranks, offsets,
+// statistics; see load_stats_kernel).
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// hist_rank
+// Block-wide exclusive scan of one int per thread (any multiple of 32 threads).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(HIST_THREADS) hist_rank_kernel(
-    const int32_t* __restrict__ idx, int64_t A, int K, int N, const int32_t* __restrict__ replica_slot,
-    int n_slots, int32_t* __restrict__ slot_out, int32_t* __restrict__ rank_out,
-    int32_t* __restrict__ blk_counts, int64_t nblk, WsHeader* hdr, uint64_t* scan_status,
-    int64_t n_tiles) {
-    extern __shared__ int32_t wh[];  // [HIST_WARPS][n_slots]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t blk = blockIdx.x;
-
-    // this call's scan state starts clean (the scan runs after this kernel)
-    if (blk == 0) {
-        for (int64_t i = threadIdx.x; i < n_tiles; i += blockDim.x) scan_status[i] = 0;
-        if (threadIdx.x == 0) { hdr->scan_ticket = 0; hdr->scan_err = 0; }
-    }
-    for (int i = threadIdx.x; i < HIST_WARPS * n_slots; i += blockDim.x) wh[i] = 0;
-    __syncthreads();
-
-    int32_t* my = wh + warp * n_slots;
-    constexpr int CH = HIST_ITEMS_PER_WARP / 32;
-    int slot_r[CH], rank_r[CH];
-    const int64_t base_a = blk * HIST_BLOCK + (int64_t)warp * HIST_ITEMS_PER_WARP;
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-        const int64_t a = base_a + j * 32 + lane;
-        int slot = -1;
-        if (a < A) {
-            int e = __ldg(idx + a);
-            if (e < 0 || e >= N) {
-                atomicOr(&hdr->scan_err, 2);  // invalid expert id: not counted
-            } else {
-                slot = e;
-                if (replica_slot != nullptr) {
-                    const int r = __ldg(replica_slot + e);
-                    const int64_t t = a / K;
-                    if (r >= 0 && (t & 1)) slot = r;
-                    if (slot >= n_slots) { atomicOr(&hdr->scan_err, 2); slot = -1; }
-                }
-            }
-            if (slot_out != nullptr) slot_out[a] = slot;
-        }
-        const unsigned peers = __match_any_sync(FULL, slot);
-        const int before = __popc(peers & lanemask_lt());
-        const int seen = (slot >= 0) ? my[slot] : 0;
-        __syncwarp();
-        if (slot >= 0 && before == 0) my[slot] = seen + __popc(peers);
-        __syncwarp();
-        slot_r[j] = slot;
-        rank_r[j] = seen + before;
-    }
-    __syncthreads();
-    // per slot: exclusive prefix over warps (stable order) and the block total
-    for (int e = threadIdx.x; e < n_slots; e += blockDim.x) {
-        int run = 0;
-#pragma unroll
-        for (int w = 0; w < HIST_WARPS; ++w) {
-            const int c = wh[w * n_slots + e];
-            wh[w * n_slots + e] = run;
-            run += c;
-        }
-        blk_counts[(int64_t)e * nblk + blk] = run;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-        const int64_t a = base_a + j * 32 + lane;
-        if (a < A) rank_out[a] = slot_r[j] >= 0 ? rank_r[j] + my[slot_r[j]] : -1;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Decoupled look-back exclusive scan (single pass).  Tile status words pack
-// (flag << 32) | value: flag 1 = tile aggregate, flag 2 = inclusive prefix.
-// Tiles are taken from a ticket counter so a tile only ever waits on tiles
-// already held by running blocks.
-// ---------------------------------------------------------------------------
-constexpr uint64_t FLAG_AGG = 1ull << 32, FLAG_PREFIX = 2ull << 32;
-
 __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* sm /*[33]*/) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -133,96 +50,339 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* sm /
     return warp_excl + x - v;
 }
 
-__global__ void __launch_bounds__(SCAN_THREADS) scan_lookback_kernel(
-    const int32_t* __restrict__ in, int32_t* __restrict__ out, int64_t L, uint64_t* status,
-    WsHeader* hdr) {
-    __shared__ int sm[33];
-    __shared__ uint32_t s_tile;
-    __shared__ int s_prefix;
-    if (threadIdx.x == 0) s_tile = atomicAdd(&hdr->scan_ticket, 1u);
-    __syncthreads();
-    const int64_t tile = s_tile;
-    const int64_t base = tile * SCAN_TILE + (int64_t)threadIdx.x * SCAN_ITEMS;
-    int v[SCAN_ITEMS];
-    int sum = 0;
+__device__ double block_sum_d(double v, double* sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-    for (int i = 0; i < SCAN_ITEMS; ++i) {
-        v[i] = (base + i < L) ? __ldg(in + base + i) : 0;
-        sum += v[i];
-    }
-    int total;
-    const int excl = block_exclusive_scan(sum, total, sm);
-    if (threadIdx.x == 0) {
-        int prefix = 0;
-        if (tile == 0) {
-            st_release_u64(status, FLAG_PREFIX | (uint32_t)total);
-        } else {
-            st_release_u64(status + tile, FLAG_AGG | (uint32_t)total);
-            int64_t p = tile - 1;
-            uint64_t t0 = 0;
-            bool timed_out = false;
-            while (p >= 0) {
-                const uint64_t s = ld_acquire_u64(status + p);
-                const uint64_t flag = s & (3ull << 32);
-                if (flag == 0) {
-                    if (t0 == 0) t0 = globaltimer();
-                    else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
-                    __nanosleep(64);
-                    continue;
-                }
-                prefix += (int)(uint32_t)s;
-                if (flag == FLAG_PREFIX) break;
-                --p;
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    __syncthreads();
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    double r = 0.0;
+    for (int w = 0; w < nw; ++w) r += sm[w];  // same order in every thread
+    return r;
+}
+
+__device__ double block_max_d(double v, double* sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmax(v, __shfl_xor_sync(FULL, v, o));
+    __syncthreads();
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    double r = sm[0];
+    for (int w = 1; w < nw; ++w) r = fmax(r, sm[w]);
+    return r;
+}
+
+__device__ __forceinline__ int ld_volatile(const int32_t* p) { return *reinterpret_cast<const volatile int32_t*>(p); }
+
+// ---------------------------------------------------------------------------
+// Single-pass load statistics.
+//
+// Each block takes the next ticket b and the assignments [b*2048, (b+1)*2048).
+//  1. slot of every assignment (replica remap), warp-private shared-memory
+//     histograms and the stable rank of each assignment inside its warp's
+//     chunk run (__match_any_sync: peers with the same slot, rank = peers
+//     before me + what the warp saw earlier);
+//  2. per-slot prefix over the block's warps and the block's slot counts,
+//     published as the block aggregate (flag 1);
+//  3. decoupled look-back over earlier blocks' vectors (aggregate or
+//     inclusive prefix) gives, per slot, the count of all earlier
+//     assignments; the block publishes its inclusive prefix (flag 2);
+//  4. rank = earlier blocks + earlier warps + within the warp: the
+//     assignment's place in its slot's segment;
+//  5. the last block to finish turns the totals into counts, offsets
+//     (exclusive scan over slots) and the statistics.
+// Every spin is bounded; on expiry the error bit is set and the kernel goes on.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void write_stats(const int (&c8)[LS_SLOTS_PER_THREAD], int total_i, int n_slots,
+                                         ScanCtl* ctl, moe_stats* stats, const double* __restrict__ hs_partial,
+                                         int hs_blocks, int N, int64_t T, double* s_red) {
+    const int tid = threadIdx.x;
+    double mx = 0.0;
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j)
+        if (tid * LS_SLOTS_PER_THREAD + j < n_slots) mx = fmax(mx, (double)c8[j]);
+    const double total = (double)total_i;
+    mx = block_max_d(mx, s_red);
+    const double mean = n_slots > 0 ? total / (double)n_slots : 0.0;
+    double var = 0.0, H = 0.0;
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid * LS_SLOTS_PER_THREAD + j;
+        if (e < n_slots) {
+            const double c = (double)c8[j];
+            var += (c - mean) * (c - mean);
+            if (c > 0.0) {
+                const double pr = c / total;
+                H -= pr * log2(pr);
             }
-            if (timed_out) atomicOr(&hdr->scan_err, 1);
-            // publish even on a timeout so later tiles do not wait in turn
-            st_release_u64(status + tile, FLAG_PREFIX | (uint32_t)(prefix + total));
         }
-        s_prefix = prefix;
     }
-    __syncthreads();
-    int run = s_prefix + excl;
-#pragma unroll
-    for (int i = 0; i < SCAN_ITEMS; ++i) {
-        if (base + i < L) out[base + i] = run;
-        run += v[i];
+    var = block_sum_d(var, s_red) / (double)(n_slots > 0 ? n_slots : 1);
+    H = block_sum_d(H, s_red);
+    double Hs = NAN;
+    if (hs_partial != nullptr) {
+        double h = 0.0;
+        for (int e = tid; e < N; e += LS_THREADS) {
+            double m = 0.0;
+            for (int q = 0; q < hs_blocks; ++q) m += hs_partial[(int64_t)q * N + e];
+            m /= (double)T;
+            if (m > 0.0) h -= m * log2(m);
+        }
+        Hs = block_sum_d(h, s_red);
+    }
+    if (tid == 0) {
+        const int err = ld_volatile(&ctl->err);
+        stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
+        stats->n_slots = n_slots;
+        stats->total = (int64_t)total_i;
+        stats->max_load = (int64_t)mx;
+        stats->mean = mean;
+        stats->imbalance = mean > 0.0 ? mx / mean : 0.0;
+        stats->std_over_mean = mean > 0.0 ? sqrt(var) / mean : 0.0;
+        stats->entropy_load_bits = H;
+        stats->entropy_score_bits = Hs;
+        stats->capacity_fixed = mx * (double)n_slots;
+        stats->capacity_125 = 1.25 * mean;
     }
 }
 
-// ---------------------------------------------------------------------------
-// finalize: in-expert rank, offsets, counts
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) finalize_kernel(
-    const int32_t* __restrict__ slot_in, const int32_t* __restrict__ idx, const int32_t* __restrict__ replica_slot,
-    int K, int64_t A, int n_slots, int64_t nblk, const int32_t* __restrict__ blk_base,
-    int32_t* __restrict__ rank, int32_t* __restrict__ offsets, int32_t* __restrict__ counts) {
-    if (blockIdx.x == 0) {
-        for (int e = threadIdx.x; e <= n_slots; e += blockDim.x) {
-            const int off = e < n_slots ? blk_base[(int64_t)e * nblk] : (int)A;
-            offsets[e] = off;
-            if (e < n_slots) {
-                const int nxt = e + 1 < n_slots ? blk_base[(int64_t)(e + 1) * nblk] : (int)A;
-                counts[e] = nxt - off;
-            }
-        }
+
+// The last block of a call: counts, offsets, statistics; then it leaves the
+// control words zeroed for the next call (every other block is done with them).
+__device__ __forceinline__ void finish_call(ScanCtl* ctl, uint32_t* flags, int64_t nblk, const int32_t* tot,
+                                         int n_slots, int64_t A, int32_t* __restrict__ counts,
+                                         int32_t* __restrict__ offsets, moe_stats* stats,
+                                         const double* __restrict__ hs_partial, int hs_blocks, int N, int64_t T,
+                                         int* s_scan, double* s_red) {
+    const int tid = threadIdx.x;
+    int c8[LS_SLOTS_PER_THREAD];
+    int tsum = 0;
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid * LS_SLOTS_PER_THREAD + j;
+        c8[j] = e < n_slots ? __ldcg(tot + e) : 0;
     }
-    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A;
-         a += (int64_t)gridDim.x * blockDim.x) {
-        int slot;
-        if (slot_in != nullptr) {
-            slot = slot_in[a];
-        } else {
-            slot = idx[a];
-            if (replica_slot != nullptr && slot >= 0) {
-                const int r = replica_slot[slot];
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) tsum += c8[j];
+    int total_i;
+    int run = block_exclusive_scan(tsum, total_i, s_scan);
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid * LS_SLOTS_PER_THREAD + j;
+        if (e < n_slots) {
+            offsets[e] = run;
+            counts[e] = c8[j];
+        }
+        run += c8[j];
+    }
+    if (tid == 0) offsets[n_slots] = (int)A;
+    if (stats != nullptr) write_stats(c8, total_i, n_slots, ctl, stats, hs_partial, hs_blocks, N, T, s_red);
+    // ready for the next call: finished count and ticket back to zero, a new
+    // epoch (this call's flags become stale), this call's errors folded into
+    // the sticky word
+    __syncthreads();
+    if (tid == 0) {
+        ctl->sticky |= ctl->err;
+        ctl->err = 0;
+        ctl->done = 0;
+        ctl->ticket = 0;
+        ctl->epoch = ctl->epoch + 1;
+    }
+}
+
+
+constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
+
+__device__ __forceinline__ uint32_t flag_tag(uint32_t epoch) { return 0x80000000u | ((epoch & 0x1FFFFFFFu) << 2); }
+// state of a flag word for the call tagged `tag`: 0 unless the word carries the tag
+__device__ __forceinline__ uint32_t flag_state(uint32_t f, uint32_t tag) { return (f & ~3u) == tag ? (f & 3u) : 0u; }
+
+__global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
+    const int32_t* __restrict__ idx, int64_t A, int K, int N, const int32_t* __restrict__ replica_slot,
+    int n_slots, int32_t* __restrict__ slot_out, int32_t* __restrict__ rank_out, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, moe_stats* stats, const double* __restrict__ hs_partial, int hs_blocks,
+    int64_t T, ScanCtl* ctl, uint32_t* flags, int32_t* agg, int32_t* pre, int64_t nblk, uint32_t ticket_base) {
+    extern __shared__ int32_t sm_dyn[];
+    int32_t* wh = sm_dyn;                          // [LS_WARPS][n_slots]
+    int32_t* ex = sm_dyn + LS_WARPS * n_slots;     // [n_slots] earlier-block counts
+    __shared__ uint32_t s_b, s_tag;
+    __shared__ int s_last;
+    __shared__ int s_scan[33];
+    __shared__ int s_win[3];
+    __shared__ double s_red[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        s_b = ticket_base + atomicAdd(&ctl->ticket, 1u);
+        s_tag = flag_tag(ld_volatile(reinterpret_cast<const int32_t*>(&ctl->epoch)));
+    }
+    for (int i = tid; i < LS_WARPS * n_slots; i += LS_THREADS) wh[i] = 0;
+    __syncthreads();
+    const int64_t b = s_b;
+    const uint32_t tag = s_tag;
+
+    // 1. slots, warp histograms, in-warp stable ranks (all loads issued first)
+    int32_t* my = wh + warp * n_slots;
+    const int64_t base_a = b * LS_BLOCK + (int64_t)warp * (LS_CHUNKS * 32);
+    int slot_r[LS_CHUNKS], rank_r[LS_CHUNKS];
+#pragma unroll
+    for (int j = 0; j < LS_CHUNKS; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        slot_r[j] = a < A ? __ldg(idx + a) : -1;
+    }
+    int bad = 0;
+#pragma unroll
+    for (int j = 0; j < LS_CHUNKS; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        int slot = slot_r[j];
+        if (a < A) {
+            if (slot < 0 || slot >= N) {
+                bad = 1;
+                slot = -1;
+            } else if (replica_slot != nullptr) {
+                const int r = __ldg(replica_slot + slot);
                 if (r >= 0 && ((a / K) & 1)) slot = r;
+                if (slot >= n_slots) { bad = 1; slot = -1; }
             }
+            if (slot_out != nullptr) slot_out[a] = slot;
         }
-        const int r = rank[a];
-        if (slot < 0 || slot >= n_slots || r < 0) continue;
-        const int64_t blk = a / HIST_BLOCK;
-        rank[a] = blk_base[(int64_t)slot * nblk + blk] - blk_base[(int64_t)slot * nblk] + r;
+        const unsigned peers = __match_any_sync(FULL, slot);
+        const int before = __popc(peers & lanemask_lt());
+        const int seen = (slot >= 0) ? my[slot] : 0;
+        __syncwarp();
+        if (slot >= 0 && before == 0) my[slot] = seen + __popc(peers);
+        __syncwarp();
+        slot_r[j] = slot;
+        rank_r[j] = seen + before;
     }
+    if (bad) atomicOr(&ctl->err, 2);
+    __syncthreads();
+
+    // 2. per-slot exclusive prefix over warps; block aggregate
+    int my_agg[LS_SLOTS_PER_THREAD];
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid + j * LS_THREADS;
+        my_agg[j] = 0;
+        if (e < n_slots) {
+            int run = 0;
+#pragma unroll
+            for (int w = 0; w < LS_WARPS; ++w) {
+                const int c = wh[w * n_slots + e];
+                wh[w * n_slots + e] = run;
+                run += c;
+            }
+            my_agg[j] = run;
+            agg[b * n_slots + e] = run;
+            if (b == 0) pre[e] = run;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release_u32(flags + b, tag | (b == 0 ? FLAG_PREFIX : FLAG_AGG));
+
+    // 3. look-back over earlier blocks, 32 at a time: warp 0 reads a window of
+    //    32 predecessor flags at once, finds the nearest inclusive prefix and
+    //    waits (bounded) only for the blocks above it to publish their
+    //    aggregates; then every thread adds, for its slots, the window's
+    //    aggregates and that prefix with independent loads.
+    int excl[LS_SLOTS_PER_THREAD];
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) excl[j] = 0;
+    if (b > 0) {
+        int64_t hi = b - 1;
+        bool timed_out = false;
+        while (hi >= 0) {
+            if (warp == 0) {
+                const int64_t p = hi - lane;
+                uint64_t t0 = 0;
+                int stop = 32, ready = 0;
+                while (true) {
+                    const uint32_t f = p >= 0 ? flag_state(ld_acquire_u32(flags + p), tag) : FLAG_PREFIX;
+                    const unsigned pm = __ballot_sync(FULL, f == FLAG_PREFIX);
+                    const unsigned zm = __ballot_sync(FULL, f == 0);
+                    stop = pm ? __ffs(pm) - 1 : 32;               // nearest prefix (lane 0 = block hi)
+                    const unsigned need = stop == 32 ? FULL : ((1u << stop) - 1u);
+                    if (!(zm & need)) { ready = 1; break; }
+                    // lane 0's clock decides for the whole warp, so the warp leaves together
+                    int give_up = 0;
+                    if (lane == 0) {
+                        if (t0 == 0) t0 = globaltimer();
+                        else give_up = globaltimer() - t0 > WAIT_LIMIT_NS;
+                    }
+                    if (__shfl_sync(FULL, give_up, 0)) break;
+                    __nanosleep(32);
+                }
+                if (lane == 0) {
+                    s_win[0] = stop;
+                    // a window that reaches below block 0 ends at the virtual prefix there
+                    s_win[1] = (stop < 32 && hi - stop >= 0) ? 1 : 0;
+                    s_win[2] = ready;
+                }
+            }
+            __syncthreads();
+            const int stop = s_win[0], has_pre = s_win[1];
+            if (!s_win[2]) timed_out = true;
+            // the window's blocks hi, hi-1, ..., hi-nagg+1 give aggregates; block
+            // hi-stop (if real) its prefix.  L2-coherent loads (ld.cg), issued
+            // eight at a time so their latencies overlap.
+            const int nagg = (int)(stop < hi + 1 ? stop : hi + 1);
+#pragma unroll
+            for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+                const int e = tid + j * LS_THREADS;
+                if (e >= n_slots) continue;
+                int acc = has_pre ? __ldcg(pre + (hi - stop) * n_slots + e) : 0;
+                for (int l0 = 0; l0 < nagg; l0 += 8) {
+                    int v8[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        v8[u] = l0 + u < nagg ? __ldcg(agg + (hi - l0 - u) * n_slots + e) : 0;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc += v8[u];
+                }
+                excl[j] += acc;
+            }
+            const bool done = stop < 32 || !s_win[2];
+            __syncthreads();  // s_win is rewritten by the next window
+            if (done) break;
+            hi -= 32;
+        }
+        if (timed_out && tid == 0) atomicOr(&ctl->err, 1);
+#pragma unroll
+        for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+            const int e = tid + j * LS_THREADS;
+            if (e < n_slots) pre[b * n_slots + e] = excl[j] + my_agg[j];
+        }
+        __threadfence();
+    }
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid + j * LS_THREADS;
+        if (e < n_slots) ex[e] = excl[j];
+    }
+    __syncthreads();
+    if (tid == 0 && b > 0) st_release_u32(flags + b, tag | FLAG_PREFIX);
+
+    // 4. in-expert ranks
+#pragma unroll
+    for (int j = 0; j < LS_CHUNKS; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        if (a < A) rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+    }
+
+    // 5. the last block to finish: counts, offsets, statistics
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    finish_call(ctl, flags, nblk, pre + (nblk - 1) * n_slots, n_slots, A, counts, offsets, stats, hs_partial,
+                hs_blocks, N, T, s_scan, s_red);
 }
 
 // ---------------------------------------------------------------------------
@@ -264,84 +424,6 @@ __global__ void __launch_bounds__(256) score_colsum_kernel(const float* __restri
         double v = 0.0;
         for (int w = 0; w < 8; ++w) v += cs[w * N + e];
         partial[(int64_t)blockIdx.x * N + e] = v;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// stats: one block
-// ---------------------------------------------------------------------------
-__device__ double block_sum_d(double v, double* sm) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    __syncthreads();
-    if (lane == 0) sm[warp] = v;
-    __syncthreads();
-    double r = 0.0;
-    for (int w = 0; w < nw; ++w) r += sm[w];  // same order in every thread
-    return r;
-}
-
-__device__ double block_max_d(double v, double* sm) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v = fmax(v, __shfl_xor_sync(FULL, v, o));
-    __syncthreads();
-    if (lane == 0) sm[warp] = v;
-    __syncthreads();
-    double r = sm[0];
-    for (int w = 1; w < nw; ++w) r = fmax(r, sm[w]);
-    return r;
-}
-
-__global__ void __launch_bounds__(1024) stats_kernel(const int32_t* __restrict__ counts, int n_slots,
-                                                     const double* __restrict__ partial, int n_part,
-                                                     int N, int64_t T, const WsHeader* hdr,
-                                                     moe_stats* out) {
-    __shared__ double sm[32];
-    double tot = 0.0, mx = 0.0;
-    for (int e = threadIdx.x; e < n_slots; e += blockDim.x) {
-        tot += (double)counts[e];
-        mx = fmax(mx, (double)counts[e]);
-    }
-    tot = block_sum_d(tot, sm);
-    mx = block_max_d(mx, sm);
-    const double mean = n_slots > 0 ? tot / (double)n_slots : 0.0;
-    double var = 0.0, H = 0.0;
-    for (int e = threadIdx.x; e < n_slots; e += blockDim.x) {
-        const double c = (double)counts[e];
-        var += (c - mean) * (c - mean);
-        if (c > 0.0) {
-            const double p = c / tot;
-            H -= p * log2(p);
-        }
-    }
-    var = block_sum_d(var, sm) / (double)(n_slots > 0 ? n_slots : 1);
-    H = block_sum_d(H, sm);
-    double Hs = NAN;
-    if (partial != nullptr) {
-        double h = 0.0;
-        for (int e = threadIdx.x; e < N; e += blockDim.x) {
-            double m = 0.0;
-            for (int b = 0; b < n_part; ++b) m += partial[(int64_t)b * N + e];
-            m /= (double)T;
-            if (m > 0.0) h -= m * log2(m);
-        }
-        Hs = block_sum_d(h, sm);
-    }
-    if (threadIdx.x == 0) {
-        const int err = hdr->scan_err;
-        out->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
-        out->n_slots = n_slots;
-        out->total = (int64_t)tot;
-        out->max_load = (int64_t)mx;
-        out->mean = mean;
-        out->imbalance = mean > 0.0 ? mx / mean : 0.0;
-        out->std_over_mean = mean > 0.0 ? sqrt(var) / mean : 0.0;
-        out->entropy_load_bits = H;
-        out->entropy_score_bits = Hs;
-        out->capacity_fixed = mx * (double)n_slots;
-        out->capacity_125 = 1.25 * mean;
     }
 }
 
@@ -390,57 +472,66 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
                               void* ws, cudaStream_t st) {
     const WsLayout L = ws_layout(T, K, N, n_slots);
     char* w = static_cast<char*>(ws);
-    WsHeader* hdr = reinterpret_cast<WsHeader*>(w + L.header);
-    int32_t* blk_counts = reinterpret_cast<int32_t*>(w + L.blk_counts);
-    int32_t* blk_base = reinterpret_cast<int32_t*>(w + L.blk_base);
-    uint64_t* status = reinterpret_cast<uint64_t*>(w + L.scan_status);
+    ScanCtl* ctl = reinterpret_cast<ScanCtl*>(w + L.ctl);
+    uint32_t* flags = reinterpret_cast<uint32_t*>(w + L.flags);
+    int32_t* agg = reinterpret_cast<int32_t*>(w + L.agg);
+    int32_t* pre = reinterpret_cast<int32_t*>(w + L.pre);
     double* partial = reinterpret_cast<double*>(w + L.hs_partial);
     const int64_t A = T * K;
-
-    const size_t hsm = sizeof(int32_t) * HIST_WARPS * (size_t)n_slots;
     cudaError_t e;
-    if (hsm > 48 * 1024) {
-        e = cudaFuncSetAttribute(hist_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm);
-        if (e != cudaSuccess) return e;
-    }
-    hist_rank_kernel<<<(unsigned)L.nblk, HIST_THREADS, hsm, st>>>(
-        idx, A, K, N, replica_slot, n_slots, slot_idx, rank, blk_counts, L.nblk, hdr, status, L.n_tiles);
-    moe_host::note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    scan_lookback_kernel<<<(unsigned)L.n_tiles, SCAN_THREADS, 0, st>>>(blk_counts, blk_base, L.L,
-                                                                       status, hdr);
-    moe_host::note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    long long fb = (A + 255) / 256;
-    const long long cap = (long long)moe_host::sm_count() * 8;
-    if (fb > cap) fb = cap;
-    if (fb < 1) fb = 1;
-    finalize_kernel<<<(unsigned)fb, 256, 0, st>>>(slot_idx, idx, replica_slot, K, A, n_slots, L.nblk,
-                                                  blk_base, rank, offsets, counts);
-    moe_host::note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    if (stats != nullptr) {
-        const double* part = nullptr;
-        if (scores != nullptr) {
-            const size_t csm = sizeof(double) * 8 * (size_t)N;
-            if (csm > 48 * 1024) {
-                e = cudaFuncSetAttribute(score_colsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)csm);
-                if (e != cudaSuccess) return e;
-            }
-            score_colsum_kernel<<<HS_BLOCKS, 256, csm, st>>>(scores, T, N, score_fn, partial);
-            moe_host::note_launch();
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            part = partial;
+    const double* part = nullptr;
+    if (stats != nullptr && scores != nullptr && T > 0) {
+        const size_t csm = sizeof(double) * 8 * (size_t)N;
+        if (csm > 48 * 1024) {
+            e = cudaFuncSetAttribute(score_colsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csm);
+            if (e != cudaSuccess) return e;
         }
-        stats_kernel<<<1, 1024, 0, st>>>(counts, n_slots, part, HS_BLOCKS, N, T, hdr, stats);
+        score_colsum_kernel<<<HS_BLOCKS, 256, csm, st>>>(scores, T, N, score_fn, partial);
         moe_host::note_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        part = partial;
     }
-    return cudaSuccess;
+    const size_t lsm = sizeof(int32_t) * (LS_WARPS + 1) * (size_t)n_slots;
+    if (lsm > 48 * 1024) {
+        e = cudaFuncSetAttribute(load_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm);
+        if (e != cudaSuccess) return e;
+    }
+    load_stats_kernel<<<(unsigned)L.nblk, LS_THREADS, lsm, st>>>(idx, A, K, N, replica_slot, n_slots, slot_idx, rank,
+                                                                  counts, offsets, stats, part, HS_BLOCKS, T, ctl,
+                                                                  flags, agg, pre, L.nblk, 0u);
+    moe_host::note_launch();
+    return cudaGetLastError();
+}
+
+// Self-test of the bounded look-back wait: a two-block problem (no
+// assignments, 8 slots) of which only the second block is launched, so the
+// flag of block 0 is never set.  The block must give up after the wait limit,
+// set the timeout bit and finish.  Returns the error bits read back.
+cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t st) {
+    const WsLayout L = ws_layout(2 * LS_BLOCK, 1, 8, 8);
+    char* w = static_cast<char*>(ws);
+    ScanCtl* ctl = reinterpret_cast<ScanCtl*>(w + L.ctl);
+    // ticket, finished count and error words start at zero; the epoch stays,
+    // so flags left by earlier calls are stale for the probe
+    cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    load_stats_kernel<<<1, LS_THREADS, sizeof(int32_t) * (LS_WARPS + 1) * 8, st>>>(
+        nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,
+        reinterpret_cast<uint32_t*>(w + L.flags), reinterpret_cast<int32_t*>(w + L.agg),
+        reinterpret_cast<int32_t*>(w + L.pre), /*nblk=*/2, /*ticket_base=*/1u);
+    moe_host::note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ScanCtl h;
+    if ((e = cudaMemcpyAsync(&h, ctl, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+    *err_out = h.err;
+    // leave the workspace as a finished call does: counters zero, next epoch
+    // (the probe's own flag becomes stale)
+    ScanCtl z;
+    memset(&z, 0, sizeof(z));
+    z.epoch = h.epoch + 1;
+    if ((e = cudaMemcpyAsync(ctl, &z, sizeof(z), cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
+    return cudaStreamSynchronize(st);
 }
 
 cudaError_t launch_replica_plan(const int32_t* counts, int N, int R, int32_t* replica_slot, cudaStream_t st) {

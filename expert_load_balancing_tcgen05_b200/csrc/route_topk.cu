@@ -14,18 +14,10 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "select.cuh"
 
 namespace moe {
 
-struct Cand {
-    float key;
-    int idx;
-    float s;
-};
-
-__device__ __forceinline__ bool beats(float ka, int ia, float kb, int ib) {
-    return (ka > kb) || (ka == kb && ia < ib);
-}
 
 // Warp-wide argmax over lanes [base, base+width) by (key desc, idx asc);
 // `width` a power of two; all lanes of the span end with the winner.
@@ -134,6 +126,190 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Filtered selection: S = N/32 threads per token, thread j owning experts
+// [32j, 32j+32) (with groups: exactly one group of 32).
+//   1. each thread: keys = fp32(s + b) of its 32 experts and their four
+//      largest (t1 >= t2 >= t3 >= t4); with groups, the group score
+//      fp32(t1 + t2) (or t1);
+//   2. group ranks by shuffles among the token's S threads; non-kept groups
+//      drop out;
+//   3. theta = the smallest t2 over the candidate threads (2 known keys
+//      each, 2 * candidate threads >= K); if too many keys pass it (a few
+//      groups holding most large keys), the K-th largest of the candidate
+//      threads' four largest keys instead.  Either way at least K candidate
+//      keys are >= theta, so the K best keys are all >= theta;
+//   4. keys >= theta (typically about ten per token) are compacted into a
+//      per-token shared-memory list, in expert order (thread-major, then
+//      ascending index), and the token's leader thread keeps the best K with
+//      the sorted 8-entry list.  A token with more survivors than its list
+//      holds (32, or 16 for N = 64) takes a slow path: its leader re-reads
+//      the whole row.
+// The result equals the plain definition: the set of keys >= theta contains
+// the top K of the candidates, and the list's order is (key desc, index asc).
+// ---------------------------------------------------------------------------
+constexpr int SEL_THREADS = 256;
+
+template <int S>
+__global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
+    const float* __restrict__ scores, const float* __restrict__ bias, int T, int K, int grouped,
+    int topk_groups, int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w) {
+    constexpr int N = 32 * S;
+    constexpr int TPB = SEL_THREADS / S;  // tokens per block
+    constexpr int SEL_CAP = S >= 4 ? 32 : 16;  // survivors kept per token in shared memory
+    __shared__ float bias_s[N];
+    __shared__ float c_key[TPB][SEL_CAP], c_s[TPB][SEL_CAP];
+    __shared__ int c_idx[TPB][SEL_CAP];
+    for (int i = threadIdx.x; i < N; i += blockDim.x) bias_s[i] = bias != nullptr ? bias[i] : 0.f;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int j = threadIdx.x % S;                 // which 32 experts
+    const int lt = threadIdx.x / S;                // token slot in the block
+    const int seg = lane - (lane % S);             // first lane of this token's segment
+    const float* bj = bias_s + 32 * j;
+
+    for (int64_t t0 = (int64_t)blockIdx.x * TPB; t0 < T; t0 += (int64_t)gridDim.x * TPB) {
+        const int64_t t = t0 + lt;
+        const bool live = t < T;
+        float s[32];
+        if (live) {
+            const float4* src = reinterpret_cast<const float4*>(scores + t * N + 32 * j);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 f = __ldg(src + q);
+                s[4 * q] = f.x; s[4 * q + 1] = f.y; s[4 * q + 2] = f.z; s[4 * q + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[i] = 0.f;
+        }
+        // 1. four largest keys of my 32 experts (a sorted, branch-free insertion)
+        float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float key = __fadd_rn(s[i], bj[i]);
+            const bool g1 = key > t1, g2 = key > t2, g3 = key > t3, g4 = key > t4;
+            t4 = g3 ? t3 : (g4 ? key : t4);
+            t3 = g2 ? t2 : (g3 ? key : t3);
+            t2 = g1 ? t1 : (g2 ? key : t2);
+            t1 = g1 ? key : t1;
+        }
+        // 2. group ranks among the token's S threads
+        bool cand = true;
+        if (grouped) {
+            const float gs = group_topn == 1 ? t1 : __fadd_rn(t1, t2);
+            int rank = 0;
+#pragma unroll
+            for (int h = 0; h < S; ++h) {
+                const float gh = __shfl_sync(FULL, gs, seg + h);
+                rank += (h != j && beats(gh, h, gs, j)) ? 1 : 0;
+            }
+            cand = rank < topk_groups;
+        }
+        // 3. theta, cheaply: the smallest t2 over the candidate threads (2 known
+        //    keys each).  Tokens whose survivors would not fit the list (a few
+        //    groups holding most large keys) tighten it to the K-th largest of
+        //    the candidate threads' four largest keys, ranked by shuffles.
+        float th = cand ? t2 : INFINITY;
+#pragma unroll
+        for (int o = 1; o < S; o <<= 1) th = fminf(th, __shfl_xor_sync(FULL, th, o));
+        unsigned m = 0;
+        if (cand) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m |= (__fadd_rn(s[i], bj[i]) >= th ? 1u : 0u) << i;
+        }
+        int total = __popc(m);
+#pragma unroll
+        for (int o = 1; o < S; o <<= 1) total += __shfl_xor_sync(FULL, total, o);
+        if (__any_sync(FULL, total > SEL_CAP && (int64_t)t < T)) {
+            const bool tighten = total > SEL_CAP;
+            float mine[4] = {cand ? t1 : -INFINITY, cand ? t2 : -INFINITY, cand ? t3 : -INFINITY,
+                             cand ? t4 : -INFINITY};
+            int rk[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int h = 0; h < S; ++h) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float u = __shfl_sync(FULL, mine[q], seg + h);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        rk[r] += (u > mine[r] || (u == mine[r] && (h * 4 + q) < (j * 4 + r))) ? 1 : 0;
+                }
+            }
+            float th2 = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                if (rk[r] == K - 1) th2 = mine[r];
+#pragma unroll
+            for (int o = 1; o < S; o <<= 1) th2 = fmaxf(th2, __shfl_xor_sync(FULL, th2, o));
+            if (tighten) {
+                th = th2;
+                m = 0;
+                if (cand) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) m |= (__fadd_rn(s[i], bj[i]) >= th ? 1u : 0u) << i;
+                }
+            }
+            total = __popc(m);
+#pragma unroll
+            for (int o = 1; o < S; o <<= 1) total += __shfl_xor_sync(FULL, total, o);
+        }
+        // 4. survivors: offsets within the token (thread order), compaction
+        const int cnt = __popc(m);
+        int off = cnt;
+#pragma unroll
+        for (int o = 1; o < S; o <<= 1) {
+            const int y = __shfl_up_sync(FULL, off, o, S);
+            if (j >= o) off += y;
+        }
+        off -= cnt;
+        if (total <= SEL_CAP) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if ((m >> i) & 1u) {
+                    c_key[lt][off] = __fadd_rn(s[i], bj[i]);
+                    c_s[lt][off] = s[i];
+                    c_idx[lt][off] = 32 * j + i;
+                    ++off;
+                }
+            }
+        }
+        // group keep bits of the token (for the slow path)
+        const unsigned keepbits = (__ballot_sync(FULL, cand) >> seg) & ((1u << S) - 1u);
+        __syncwarp();
+        if (j == 0 && live) {
+            Top8 top;
+            top.init();
+            if (total <= SEL_CAP) {
+                for (int c = 0; c < total; ++c) top.offer(c_key[lt][c], c_idx[lt][c], c_s[lt][c]);
+            } else {
+                const float* row = scores + t * N;
+                for (int e = 0; e < N; ++e) {
+                    if (!((keepbits >> (e >> 5)) & 1u)) continue;
+                    const float sv = row[e];
+                    const float key = __fadd_rn(sv, bias_s[e]);
+                    if (key >= th) top.offer(key, e, sv);
+                }
+            }
+            top.write(K, renorm, route_scale, topk_idx + t * K, topk_w + t * K);
+        }
+        __syncwarp();
+    }
+}
+
+// The filtered kernel covers N in {64, 128, 256}, K <= 8, and either one
+// group or groups of exactly 32 experts with a group score of the top one or
+// two keys, when the candidate threads hold at least K known keys (2 each).
+static bool select_fast_ok(int N, int K, int n_groups, int topk_groups, int group_topn) {
+    if (!(N == 64 || N == 128 || N == 256) || K > 8) return false;
+    const int S = N / 32;
+    if (n_groups == 1) return 2 * S >= K;
+    return N / n_groups == 32 && group_topn >= 1 && group_topn <= 2 && 2 * topk_groups >= K;
+}
+
 // Elements per lane for N experts; 0 if unsupported.
 int route_epl(int N) {
     if (N <= 32) return 1;
@@ -147,6 +323,24 @@ int route_epl(int N) {
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K,
                               int n_groups, int topk_groups, int group_topn, int renorm,
                               float route_scale, int32_t* idx, float* w, cudaStream_t st) {
+    if (select_fast_ok(N, K, n_groups, topk_groups, group_topn)) {
+        const int S = N / 32;
+        long long blocks = ((long long)T * S + SEL_THREADS - 1) / SEL_THREADS;
+        const long long cap = (long long)moe_host::sm_count() * 16;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+        const int grouped = n_groups > 1 ? 1 : 0;
+        switch (S) {
+            case 2: route_select_kernel<2><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
+                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
+            case 4: route_select_kernel<4><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
+                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
+            default: route_select_kernel<8><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
+                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
+        }
+        moe_host::note_launch();
+        return cudaGetLastError();
+    }
     const int epl = route_epl(N);
     const int gsize = N / n_groups;
     const int lpg = n_groups > 1 ? gsize / epl : 32;

@@ -28,7 +28,7 @@ MOE_F32, MOE_BF16 = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
-           "moe_version", "moe_load_stats_noalloc")
+           "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout")
 
 
 class RouteCfg(ctypes.Structure):
@@ -149,6 +149,14 @@ def moe_dispatch(x, T, d, K, slot_idx, offsets, rank, rows, rows_fp8, scales, po
 def moe_combine(y, T, d, K, pos, w, out, stream=None):
     _check(_lib.moe_combine(_ptr(y), _dtype_code(y), T, d, K, _ptr(pos), _ptr(w), _ptr(out), _stream(stream)),
            "moe_combine")
+
+
+_lib.moe_selftest_wait_timeout.argtypes = [_P, _SZ, _P]
+_lib.moe_selftest_wait_timeout.restype = _I32
+
+
+def moe_selftest_wait_timeout(ws, stream=None) -> int:
+    return int(_lib.moe_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_workspace_status(ws, stream=None) -> int:

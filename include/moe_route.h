@@ -15,9 +15,9 @@
  *    MOE_ERR_CUDA.  Nothing aborts or traps.
  *  - Device-side waits (TMA/MMA barriers in the gate GEMM, the look-back of
  *    the offsets scan) are bounded.  A wait that runs out sets an error word
- *    in the workspace and the kernel returns early; read it with
- *    moe_workspace_status().  The load-statistics struct also carries the
- *    scan's status of that call.
+ *    in the workspace (sticky until read) and the kernel returns early; read
+ *    it with moe_workspace_status().  The load-statistics struct also
+ *    carries the status of its own call.
  *  - 16-byte alignment is required for x, w_gate, rows, y and out.
  *  - Flat assignment counts must satisfy T*K < 2^31.
  *
@@ -93,7 +93,8 @@ typedef struct {
 /* Bytes of workspace the calls below need for T tokens, K choices, N experts
  * and n_slots histogram slots (n_slots >= N; N + replicas).  One workspace
  * may serve every call on one stream; calls that overlap on the GPU need
- * their own workspaces.  Contents need no initialisation. */
+ * their own workspaces.  Zero-fill it once before its first use; every call
+ * leaves it ready for the next one, so no per-call initialisation is needed. */
 size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
 
 /*
@@ -108,6 +109,12 @@ size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
  * Scores, fused into the GEMM epilogue, written to scores [T,N] fp32:
  *   softmax over N ([ENT] softmax equation) or sigmoid ([HD] "Token routing").
  *   If x == NULL the call skips the GEMM and reads `scores` as input instead.
+ *   With bf16 inputs, N in {64, 128, 256}, K <= 8 and either one group or
+ *   sigmoid scores in groups of 32 experts with group_topn <= 2, the
+ *   selection below can also run inside the GEMM epilogue (no scores round
+ *   trip); `scores` may then be NULL, and with `scores` given the library
+ *   picks the faster of the two for the batch size (environment variable
+ *   MOE_FUSED_SELECT=0/1 forces one).  Otherwise `scores` is required.
  * Selection ([HD] "Auxiliary-loss-free load balancing": the bias steers only
  * the choice; [GL] sections 1 and 3: group-limited routing):
  *   key = fp32(s + bias) (bias [N] fp32 or NULL); with n_groups > 1 the
@@ -141,8 +148,11 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
  * stats (device, may be NULL): see moe_stats.  scores [T,N] fp32 (may be
  *   NULL) adds entropy_score_bits, with score_fn telling softmax rows
  *   (used as they are) from sigmoid rows (normalised per token).
- * Offsets come from a single-pass decoupled look-back scan over per-block
- * counts; its waits are bounded (stats->status = MOE_ERR_TIMEOUT on expiry).
+ * One single-pass kernel: blocks of 2048 assignments publish their per-slot
+ * counts and look back over earlier blocks' count vectors (decoupled
+ * look-back) for the ranks; the last block to finish writes counts, offsets
+ * and stats.  Its waits are bounded (stats->status = MOE_ERR_TIMEOUT on
+ * expiry).
  */
 moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
                           const int32_t* replica_slot, int32_t n_slots, int32_t* slot_idx,
@@ -236,10 +246,19 @@ moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T, int32_t K,
                                   const float* scores, int32_t score_fn, moe_stats* stats,
                                   moe_stream_t stream);
 
-/* Synchronises `stream`, reads and clears the workspace's device error
- * words: MOE_OK, or MOE_ERR_TIMEOUT if a bounded wait ran out since the last
- * check.  (The only call that synchronises.) */
+/* Synchronises `stream`, reads and clears the workspace's sticky device
+ * error words: MOE_OK, MOE_ERR_TIMEOUT if a bounded wait ran out, or
+ * MOE_ERR_INVALID if an expert id was out of range, since the last check.
+ * (The calls that synchronise are this one and moe_selftest_wait_timeout.) */
 moe_status moe_workspace_status(void* ws, moe_stream_t stream);
+
+/* Self-test of the bounded device waits: runs the offsets pass's look-back
+ * on a two-block problem where the flag it waits for is never set.  The wait
+ * must give up after about one second, record the timeout and return, and the
+ * CUDA context stays usable.  Returns MOE_ERR_TIMEOUT when the wait ran out as
+ * designed (the expected result), MOE_OK if it did not.  Synchronises
+ * `stream`; ws needs moe_workspace_bytes(4096, 1, 8, 8) bytes. */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Kernel launches issued by this library on the calling thread since the
  * last reset (for launch accounting). */

@@ -253,4 +253,21 @@ def test_launch_count_counts_kernels():
     idx = W.make_assignments(T, K, N, seed=1).cuda()
     moe.moe_launch_count(reset=True)
     load_stats_gpu(idx, T, K, N)
-    assert moe.moe_launch_count() == 4  # hist, scan, finalize, stats
+    assert moe.moe_launch_count() == 1  # one single-pass kernel
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """The look-back wait of the offsets pass, run on a flag nothing sets,
+    gives up after about a second with a timeout status; the context stays
+    usable for the next call."""
+    import time
+    moe = lib()
+    ws = moe.workspace(4096, 1, 8)
+    t0 = time.time()
+    assert moe.moe_selftest_wait_timeout(ws) == moe.MOE_ERR_TIMEOUT
+    assert 0.5 < time.time() - t0 < 30
+    T, K, N = 300, 4, 16
+    idx = W.make_assignments(T, K, N, seed=5).cuda()
+    _, counts, _, _, stats, ws2 = load_stats_gpu(idx, T, K, N)
+    assert lib().read_stats(stats)["status"] == 0
+    assert int(counts.sum()) == T * K

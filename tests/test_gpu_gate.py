@@ -27,6 +27,14 @@ def _check_scores(s_gpu, s_ref):
     assert not bad.any(), (int(bad.sum()), float(err.max()))
 
 
+@pytest.fixture(params=["separate", "fused"], autouse=True)
+def select_path(request, monkeypatch):
+    """Run every case with the selection in its own kernel and inside the
+    GEMM epilogue (where the configuration allows it)."""
+    monkeypatch.setenv("MOE_FUSED_SELECT", "0" if request.param == "separate" else "1")
+    return request.param
+
+
 def _run_and_check(orc, wl, T, d, seed, check_gap=True):
     wl = wl.with_(T=T, d=d)
     inp = W.make_inputs(wl, seed=seed)
@@ -99,3 +107,45 @@ def test_zero_gate_gives_uniform_scores():
     assert torch.all(s == 0.5)
     # all-equal scores select the lowest experts (ties to the lower index)
     assert torch.equal(idx.cpu(), torch.arange(8, dtype=torch.int32).expand(256, 8))
+
+
+def test_fused_selection_without_scores_output():
+    """With the selection inside the GEMM epilogue the scores output is
+    optional; the choice and weights are the same with or without it."""
+    moe = lib()
+    wl = W.WORKLOADS["v3_router"].with_(T=777, d=1024)
+    inp = W.make_inputs(wl, seed=9)
+    x, Wg, b = inp["x"].cuda(), inp["W"].cuda(), inp["bias"].cuda()
+    s1, i1, w1, _ = route_gpu(wl, x, Wg, None, b)
+    i2 = torch.empty_like(i1)
+    w2 = torch.empty_like(w1)
+    ws = moe.workspace(wl.T, wl.K, wl.N)
+    cfg = moe.route_cfg(wl.T, wl.d, wl.N, wl.K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm,
+                        wl.scale)
+    moe.moe_route(cfg, x, Wg, None, b, None, i2, w2, ws)
+    assert torch.equal(i1, i2) and torch.equal(w1, w2)
+    # the non-fused configuration (groups of 16) refuses a missing scores buffer
+    cfg16 = moe.route_cfg(wl.T, wl.d, wl.N, wl.K, wl.fn, 16, 4, 2, True, 2.5)
+    with pytest.raises(moe.MoeError):
+        moe.moe_route(cfg16, x, Wg, None, b, None, i2, w2, ws)
+
+
+def test_gate_pair_many_tiles_per_cluster(orc):
+    """N = 256 runs on CTA pairs (2-SM MMA); with more 256-token tiles than
+    pairs, every pair runs several tiles and a ragged last tile."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    T = (sms // 2) * 256 * 2 + 300
+    _run_and_check(orc, W.WORKLOADS["v3_router"], T, 256, seed=12)
+
+
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_gate_one_sm_and_pair_agree(pair, monkeypatch):
+    """The 1-SM and 2-SM kernels compute the same scores up to fp32
+    accumulation order, and the same selection from them."""
+    monkeypatch.setenv("MOE_GATE_PAIR", pair)
+    wl = W.WORKLOADS["v3_router"].with_(T=1000, d=2048)
+    inp = W.make_inputs(wl, seed=13)
+    s, idx, w, ws = route_gpu(wl, inp["x"].cuda(), inp["W"].cuda(), None, inp["bias"].cuda())
+    assert lib().moe_workspace_status(ws) == 0
+    ref = inp["x"].cuda().float() @ inp["W"].cuda().float().t()
+    assert torch.allclose(s, torch.sigmoid(ref), rtol=1e-3, atol=1e-6)
