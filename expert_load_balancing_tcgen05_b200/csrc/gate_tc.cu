@@ -194,7 +194,7 @@ struct Xch {
 // grouped selection exchanges group scores; half 1 hands its top-8 to half 0,
 // which merges and writes the row's choice.  Every epilogue thread executes
 // the same sequence of epi_sync() calls.
-template <int BN>
+template <int BN, bool FUSED>
 __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int row, int h, int64_t grow,
                                              const float* off_s, const float* bias_s, const Xch& x) {
     constexpr int NC = BN / 32, NCH = NC / 2;
@@ -205,7 +205,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
     Top8 top;
     top.init();
     if (p.fn == MOE_SIGMOID) {
-        if (p.fused && p.n_groups > 1) {
+        if (FUSED && p.n_groups > 1) {
             // one expert group per 32-column chunk: group score = sum of its top-n keys
 #pragma unroll
             for (int cc = 0; cc < NCH; ++cc) {
@@ -253,7 +253,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
-                    if (p.fused) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
+                    if constexpr (FUSED) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
                 }
                 if (srow) store32(srow + 32 * c, v);
             }
@@ -289,12 +289,12 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
-                if (p.fused) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
+                if constexpr (FUSED) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
             }
             if (srow) store32(srow + 32 * c, v);
         }
     }
-    if (!p.fused) return;
+    if constexpr (!FUSED) return;
     // half 1 hands its list to half 0; its indices are all above half 0's,
     // so offering them in list order keeps (key desc, index asc)
     if (h == 1) {
@@ -309,7 +309,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
     }
 }
 
-template <int BN>
+template <int BN, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                              const __grid_constant__ CUtensorMap tmB, int d,
                                                              const Epi p, int32_t* err, int num_tiles) {
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
             fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + a * BN;
             const int64_t grow = (int64_t)tile * BM + row;
-            epilogue_row<BN>(p, taddr, row, h, grow, off_s, bias_s, xch);
+            epilogue_row<BN, FUSED>(p, taddr, row, h, grow, off_s, bias_s, xch);
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty0 + 8 * a);
@@ -526,6 +526,7 @@ __device__ __forceinline__ constexpr uint32_t idesc_pair() {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
+template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gate_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int d,
                         const Epi p, int32_t* err, int num_pairs) {
@@ -648,7 +649,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + a * BN;
             const int64_t grow = (int64_t)tp * 2 * BM + (int64_t)rank * BM + row;
-            epilogue_row<BN>(p, taddr, row, h, grow, off_s, bias_s, xch);
+            epilogue_row<BN, FUSED>(p, taddr, row, h, grow, off_s, bias_s, xch);
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * a);
@@ -719,13 +720,14 @@ static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, 256, d, tc::BM)) return cudaErrorInvalidValue;
     const size_t smem = tc::PairCfg::SMEM_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(tc::gate_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.fused ? tc::gate_tc_pair_kernel<true> : tc::gate_tc_pair_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int num_pairs = (T + 2 * tc::BM - 1) / (2 * tc::BM);
     int clusters = moe_host::sm_count() / 2;
     if (clusters > num_pairs) clusters = num_pairs;
     if (clusters < 1) clusters = 1;
-    tc::gate_tc_pair_kernel<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);
+    kern<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);
     moe_host::note_launch();
     return cudaGetLastError();
 }
@@ -736,13 +738,14 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, BN, d, BN)) return cudaErrorInvalidValue;
     const size_t smem = tc::Cfg<BN>::SMEM_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(tc::gate_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.fused ? tc::gate_tc_kernel<BN, true> : tc::gate_tc_kernel<BN, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int num_tiles = (T + tc::BM - 1) / tc::BM;
     int grid = moe_host::sm_count();
     if (grid > num_tiles) grid = num_tiles;
     if (grid < 1) grid = 1;
-    tc::gate_tc_kernel<BN><<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles);
+    kern<<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles);
     moe_host::note_launch();
     return cudaGetLastError();
 }

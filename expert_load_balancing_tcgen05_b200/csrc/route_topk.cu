@@ -130,9 +130,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 // ---------------------------------------------------------------------------
 // Filtered selection: S = N/32 threads per token, thread j owning experts
 // [32j, 32j+32) (with groups: exactly one group of 32).
-//   1. each thread: keys = fp32(s + b) of its 32 experts and their four
-//      largest (t1 >= t2 >= t3 >= t4); with groups, the group score
-//      fp32(t1 + t2) (or t1);
+//   1. each thread: keys = fp32(s + b) of its 32 experts and their two
+//      largest (t1 >= t2); with groups, the group score fp32(t1 + t2) (or t1);
 //   2. group ranks by shuffles among the token's S threads; non-kept groups
 //      drop out;
 //   3. theta = the smallest t2 over the candidate threads (2 known keys
@@ -142,10 +141,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 //      keys are >= theta, so the K best keys are all >= theta;
 //   4. keys >= theta (typically about ten per token) are compacted into a
 //      per-token shared-memory list, in expert order (thread-major, then
-//      ascending index), and the token's leader thread keeps the best K with
-//      the sorted 8-entry list.  A token with more survivors than its list
-//      holds (32, or 16 for N = 64) takes a slow path: its leader re-reads
-//      the whole row.
+//      ascending index);
+//   5. the token's threads rank the survivors in parallel (rank = how many
+//      survivors beat it in the (key desc, index asc) order) and place the K
+//      best at their ranks; the leader writes weights in k order.  A token
+//      with more survivors than its list holds (32, or 16 for N = 64) takes
+//      a slow path: its leader re-reads the whole row.
 // The result equals the plain definition: the set of keys >= theta contains
 // the top K of the candidates, and the list's order is (key desc, index asc).
 // ---------------------------------------------------------------------------
@@ -157,11 +158,13 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
     int topk_groups, int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w) {
     constexpr int N = 32 * S;
-    constexpr int TPB = SEL_THREADS / S;  // tokens per block
+    constexpr int TPB = SEL_THREADS / S;       // tokens per block
     constexpr int SEL_CAP = S >= 4 ? 32 : 16;  // survivors kept per token in shared memory
     __shared__ float bias_s[N];
     __shared__ float c_key[TPB][SEL_CAP], c_s[TPB][SEL_CAP];
     __shared__ int c_idx[TPB][SEL_CAP];
+    __shared__ float o_s[TPB][8];
+    __shared__ int o_i[TPB][8];
     for (int i = threadIdx.x; i < N; i += blockDim.x) bias_s[i] = bias != nullptr ? bias[i] : 0.f;
     __syncthreads();
 
@@ -186,16 +189,13 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[i] = 0.f;
         }
-        // 1. four largest keys of my 32 experts (a sorted, branch-free insertion)
-        float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;
+        // 1. two largest keys of my 32 experts
+        float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float key = __fadd_rn(s[i], bj[i]);
-            const bool g1 = key > t1, g2 = key > t2, g3 = key > t3, g4 = key > t4;
-            t4 = g3 ? t3 : (g4 ? key : t4);
-            t3 = g2 ? t2 : (g3 ? key : t3);
-            t2 = g1 ? t1 : (g2 ? key : t2);
-            t1 = g1 ? key : t1;
+            t2 = key > t1 ? t1 : (key > t2 ? key : t2);
+            t1 = key > t1 ? key : t1;
         }
         // 2. group ranks among the token's S threads
         bool cand = true;
@@ -224,25 +224,35 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
         int total = __popc(m);
 #pragma unroll
         for (int o = 1; o < S; o <<= 1) total += __shfl_xor_sync(FULL, total, o);
-        if (__any_sync(FULL, total > SEL_CAP && (int64_t)t < T)) {
+        if (__any_sync(FULL, total > SEL_CAP && live)) {
             const bool tighten = total > SEL_CAP;
-            float mine[4] = {cand ? t1 : -INFINITY, cand ? t2 : -INFINITY, cand ? t3 : -INFINITY,
-                             cand ? t4 : -INFINITY};
+            float q4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (cand) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float key = __fadd_rn(s[i], bj[i]);
+                    const bool g1 = key > q4[0], g2 = key > q4[1], g3 = key > q4[2], g4 = key > q4[3];
+                    q4[3] = g3 ? q4[2] : (g4 ? key : q4[3]);
+                    q4[2] = g2 ? q4[1] : (g3 ? key : q4[2]);
+                    q4[1] = g1 ? q4[0] : (g2 ? key : q4[1]);
+                    q4[0] = g1 ? key : q4[0];
+                }
+            }
             int rk[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int h = 0; h < S; ++h) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float u = __shfl_sync(FULL, mine[q], seg + h);
+                    const float u = __shfl_sync(FULL, q4[q], seg + h);
 #pragma unroll
                     for (int r = 0; r < 4; ++r)
-                        rk[r] += (u > mine[r] || (u == mine[r] && (h * 4 + q) < (j * 4 + r))) ? 1 : 0;
+                        rk[r] += (u > q4[r] || (u == q4[r] && (h * 4 + q) < (j * 4 + r))) ? 1 : 0;
                 }
             }
             float th2 = -INFINITY;
 #pragma unroll
             for (int r = 0; r < 4; ++r)
-                if (rk[r] == K - 1) th2 = mine[r];
+                if (rk[r] == K - 1) th2 = q4[r];
 #pragma unroll
             for (int o = 1; o < S; o <<= 1) th2 = fmaxf(th2, __shfl_xor_sync(FULL, th2, o));
             if (tighten) {
@@ -277,22 +287,38 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
                 }
             }
         }
-        // group keep bits of the token (for the slow path)
         const unsigned keepbits = (__ballot_sync(FULL, cand) >> seg) & ((1u << S) - 1u);
         __syncwarp();
-        if (j == 0 && live) {
+        if (total <= SEL_CAP) {
+            // 5. each of the token's threads ranks a share of the survivors; a
+            //    survivor beaten by fewer than K others is placed at its rank
+            for (int c = j; c < total; c += S) {
+                const float kc = c_key[lt][c];
+                const int ic = c_idx[lt][c];
+                int rank = 0;
+                for (int c2 = 0; c2 < total; ++c2) rank += beats(c_key[lt][c2], c_idx[lt][c2], kc, ic) ? 1 : 0;
+                if (rank < K) { o_i[lt][rank] = ic; o_s[lt][rank] = c_s[lt][c]; }
+            }
+            __syncwarp();
+            if (j == 0 && live) {
+                float ssum = o_s[lt][0];
+                for (int k = 1; k < K; ++k) ssum = __fadd_rn(ssum, o_s[lt][k]);
+                for (int k = 0; k < K; ++k) {
+                    const float wv = renorm ? __fdiv_rn(o_s[lt][k], ssum) : o_s[lt][k];
+                    topk_idx[t * K + k] = o_i[lt][k];
+                    topk_w[t * K + k] = __fmul_rn(wv, route_scale);
+                }
+            }
+        } else if (j == 0 && live) {
+            // slow path: the leader re-reads the whole row
             Top8 top;
             top.init();
-            if (total <= SEL_CAP) {
-                for (int c = 0; c < total; ++c) top.offer(c_key[lt][c], c_idx[lt][c], c_s[lt][c]);
-            } else {
-                const float* row = scores + t * N;
-                for (int e = 0; e < N; ++e) {
-                    if (!((keepbits >> (e >> 5)) & 1u)) continue;
-                    const float sv = row[e];
-                    const float key = __fadd_rn(sv, bias_s[e]);
-                    if (key >= th) top.offer(key, e, sv);
-                }
+            const float* row = scores + t * N;
+            for (int e = 0; e < N; ++e) {
+                if (!((keepbits >> (e >> 5)) & 1u)) continue;
+                const float sv = row[e];
+                const float key = __fadd_rn(sv, bias_s[e]);
+                if (key >= th) top.offer(key, e, sv);
             }
             top.write(K, renorm, route_scale, topk_idx + t * K, topk_w + t * K);
         }
