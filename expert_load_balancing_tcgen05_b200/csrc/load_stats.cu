@@ -91,79 +91,25 @@ __device__ __forceinline__ int ld_volatile(const int32_t* p) { return *reinterpr
 //     assignments; the block publishes its inclusive prefix (flag 2);
 //  4. rank = earlier blocks + earlier warps + within the warp: the
 //     assignment's place in its slot's segment;
-//  5. the last block to finish turns the totals into counts, offsets
-//     (exclusive scan over slots) and the statistics.
+//  5. the block with the last ticket turns its inclusive prefix (the
+//     totals) into counts, offsets (exclusive scan over slots) and the
+//     statistics; the last block to finish resets the control words.
 // Every spin is bounded; on expiry the error bit is set and the kernel goes on.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void write_stats(const int (&c8)[LS_SLOTS_PER_THREAD], int total_i, int n_slots,
-                                         ScanCtl* ctl, moe_stats* stats, const double* __restrict__ hs_partial,
-                                         int hs_blocks, int N, int64_t T, double* s_red) {
-    const int tid = threadIdx.x;
-    double mx = 0.0;
-#pragma unroll
-    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j)
-        if (tid * LS_SLOTS_PER_THREAD + j < n_slots) mx = fmax(mx, (double)c8[j]);
-    const double total = (double)total_i;
-    mx = block_max_d(mx, s_red);
-    const double mean = n_slots > 0 ? total / (double)n_slots : 0.0;
-    double var = 0.0, H = 0.0;
-#pragma unroll
-    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
-        const int e = tid * LS_SLOTS_PER_THREAD + j;
-        if (e < n_slots) {
-            const double c = (double)c8[j];
-            var += (c - mean) * (c - mean);
-            if (c > 0.0) {
-                const double pr = c / total;
-                H -= pr * log2(pr);
-            }
-        }
-    }
-    var = block_sum_d(var, s_red) / (double)(n_slots > 0 ? n_slots : 1);
-    H = block_sum_d(H, s_red);
-    double Hs = NAN;
-    if (hs_partial != nullptr) {
-        double h = 0.0;
-        for (int e = tid; e < N; e += LS_THREADS) {
-            double m = 0.0;
-            for (int q = 0; q < hs_blocks; ++q) m += hs_partial[(int64_t)q * N + e];
-            m /= (double)T;
-            if (m > 0.0) h -= m * log2(m);
-        }
-        Hs = block_sum_d(h, s_red);
-    }
-    if (tid == 0) {
-        const int err = ld_volatile(&ctl->err);
-        stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
-        stats->n_slots = n_slots;
-        stats->total = (int64_t)total_i;
-        stats->max_load = (int64_t)mx;
-        stats->mean = mean;
-        stats->imbalance = mean > 0.0 ? mx / mean : 0.0;
-        stats->std_over_mean = mean > 0.0 ? sqrt(var) / mean : 0.0;
-        stats->entropy_load_bits = H;
-        stats->entropy_score_bits = Hs;
-        stats->capacity_fixed = mx * (double)n_slots;
-        stats->capacity_125 = 1.25 * mean;
-    }
-}
-
-
-// The last block of a call: counts, offsets, statistics; then it leaves the
-// control words zeroed for the next call (every other block is done with them).
-__device__ __forceinline__ void finish_call(ScanCtl* ctl, uint32_t* flags, int64_t nblk, const int32_t* tot,
-                                         int n_slots, int64_t A, int32_t* __restrict__ counts,
-                                         int32_t* __restrict__ offsets, moe_stats* stats,
-                                         const double* __restrict__ hs_partial, int hs_blocks, int N, int64_t T,
-                                         int* s_scan, double* s_red) {
-    const int tid = threadIdx.x;
+// counts, offsets and statistics from the totals (the last block's
+// inclusive prefix over blocks); one combined block reduction for the stats
+__device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, int64_t A, int32_t* __restrict__ counts,
+                                              int32_t* __restrict__ offsets, moe_stats* stats,
+                                              const double* __restrict__ hs_partial, int hs_blocks, int N, int64_t T,
+                                              const ScanCtl* ctl, int* s_scan, double* s_red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int c8[LS_SLOTS_PER_THREAD];
-    int tsum = 0;
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
         const int e = tid * LS_SLOTS_PER_THREAD + j;
         c8[j] = e < n_slots ? __ldcg(tot + e) : 0;
     }
+    int tsum = 0;
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) tsum += c8[j];
     int total_i;
@@ -178,20 +124,64 @@ __device__ __forceinline__ void finish_call(ScanCtl* ctl, uint32_t* flags, int64
         run += c8[j];
     }
     if (tid == 0) offsets[n_slots] = (int)A;
-    if (stats != nullptr) write_stats(c8, total_i, n_slots, ctl, stats, hs_partial, hs_blocks, N, T, s_red);
-    // ready for the next call: finished count and ticket back to zero, a new
-    // epoch (this call's flags become stale), this call's errors folded into
-    // the sticky word
+    if (stats == nullptr) return;
+    const double total = (double)total_i;
+    const double mean = n_slots > 0 ? total / (double)n_slots : 0.0;
+    double mx = 0.0, var = 0.0, H = 0.0, Hs = 0.0;
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid * LS_SLOTS_PER_THREAD + j;
+        if (e < n_slots) {
+            const double c = (double)c8[j];
+            mx = fmax(mx, c);
+            var += (c - mean) * (c - mean);
+            if (c > 0.0) {
+                const double pr = c / total;
+                H -= pr * log2(pr);
+            }
+        }
+    }
+    if (hs_partial != nullptr) {
+        for (int e = tid; e < N; e += LS_THREADS) {
+            double m = 0.0;
+            for (int q = 0; q < hs_blocks; ++q) m += hs_partial[(int64_t)q * N + e];
+            m /= (double)T;
+            if (m > 0.0) Hs -= m * log2(m);
+        }
+    }
+    // one reduction round for (max, var, H, Hs): warp butterflies, then warp 0
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        mx = fmax(mx, __shfl_xor_sync(FULL, mx, o));
+        var += __shfl_xor_sync(FULL, var, o);
+        H += __shfl_xor_sync(FULL, H, o);
+        Hs += __shfl_xor_sync(FULL, Hs, o);
+    }
+    if (lane == 0) { s_red[warp] = mx; s_red[8 + warp] = var; s_red[16 + warp] = H; s_red[24 + warp] = Hs; }
     __syncthreads();
     if (tid == 0) {
-        ctl->sticky |= ctl->err;
-        ctl->err = 0;
-        ctl->done = 0;
-        ctl->ticket = 0;
-        ctl->epoch = ctl->epoch + 1;
+        double rmx = s_red[0], rvar = 0.0, rH = 0.0, rHs = 0.0;
+        for (int w = 0; w < LS_WARPS; ++w) {
+            rmx = fmax(rmx, s_red[w]);
+            rvar += s_red[8 + w];
+            rH += s_red[16 + w];
+            rHs += s_red[24 + w];
+        }
+        rvar /= (double)(n_slots > 0 ? n_slots : 1);
+        const int err = ld_volatile(&ctl->err);
+        stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
+        stats->n_slots = n_slots;
+        stats->total = (int64_t)total_i;
+        stats->max_load = (int64_t)rmx;
+        stats->mean = mean;
+        stats->imbalance = mean > 0.0 ? rmx / mean : 0.0;
+        stats->std_over_mean = mean > 0.0 ? sqrt(rvar) / mean : 0.0;
+        stats->entropy_load_bits = rH;
+        stats->entropy_score_bits = hs_partial != nullptr ? rHs : NAN;
+        stats->capacity_fixed = rmx * (double)n_slots;
+        stats->capacity_125 = 1.25 * mean;
     }
 }
-
 
 constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
 
@@ -208,7 +198,6 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
     int32_t* wh = sm_dyn;                          // [LS_WARPS][n_slots]
     int32_t* ex = sm_dyn + LS_WARPS * n_slots;     // [n_slots] earlier-block counts
     __shared__ uint32_t s_b, s_tag;
-    __shared__ int s_last;
     __shared__ int s_scan[33];
     __shared__ int s_win[3];
     __shared__ double s_red[32];
@@ -326,22 +315,19 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
             const int stop = s_win[0], has_pre = s_win[1];
             if (!s_win[2]) timed_out = true;
             // the window's blocks hi, hi-1, ..., hi-nagg+1 give aggregates; block
-            // hi-stop (if real) its prefix.  L2-coherent loads (ld.cg), issued
-            // eight at a time so their latencies overlap.
+            // hi-stop (if real) its prefix.  L2-coherent loads (ld.cg), all
+            // issued before the first is used: one L2 latency per window.
             const int nagg = (int)(stop < hi + 1 ? stop : hi + 1);
 #pragma unroll
             for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
                 const int e = tid + j * LS_THREADS;
                 if (e >= n_slots) continue;
+                int v32[32];
+#pragma unroll
+                for (int l = 0; l < 32; ++l) v32[l] = l < nagg ? __ldcg(agg + (hi - l) * n_slots + e) : 0;
                 int acc = has_pre ? __ldcg(pre + (hi - stop) * n_slots + e) : 0;
-                for (int l0 = 0; l0 < nagg; l0 += 8) {
-                    int v8[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        v8[u] = l0 + u < nagg ? __ldcg(agg + (hi - l0 - u) * n_slots + e) : 0;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) acc += v8[u];
-                }
+                for (int l = 0; l < 32; ++l) acc += v32[l];
                 excl[j] += acc;
             }
             const bool done = stop < 32 || !s_win[2];
@@ -372,17 +358,27 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
         if (a < A) rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
     }
 
-    // 5. the last block to finish: counts, offsets, statistics
+    // 5. the block with the last ticket holds the totals in its inclusive
+    //    prefix: it writes counts, offsets and statistics while the other
+    //    blocks still write ranks; the last block to finish resets the
+    //    control words for the next call
+    if (b == nblk - 1 && counts != nullptr) {  // (the bounded-wait self-test passes no outputs)
+        __syncthreads();
+        finish_totals(pre + b * n_slots, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T, ctl,
+                      s_scan, s_red);
+    }
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        s_last = atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1);
+        if (atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1)) {
+            __threadfence();
+            ctl->sticky |= ctl->err;
+            ctl->err = 0;
+            ctl->done = 0;
+            ctl->ticket = 0;
+            ctl->epoch = ctl->epoch + 1;
+        }
     }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    finish_call(ctl, flags, nblk, pre + (nblk - 1) * n_slots, n_slots, A, counts, offsets, stats, hs_partial,
-                hs_blocks, N, T, s_scan, s_red);
 }
 
 // ---------------------------------------------------------------------------
@@ -524,9 +520,9 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
     ScanCtl h;
     if ((e = cudaMemcpyAsync(&h, ctl, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return e;
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
-    *err_out = h.err;
+    *err_out = h.err | h.sticky;  // the probe's block is also the last to finish: it folds err into sticky
     // leave the workspace as a finished call does: counters zero, next epoch
-    // (the probe's own flag becomes stale)
+    // (the probe's own flag becomes stale), error words cleared
     ScanCtl z;
     memset(&z, 0, sizeof(z));
     z.epoch = h.epoch + 1;

@@ -257,7 +257,8 @@ moe_status moe_workspace_status(void* ws, moe_stream_t stream);
  * must give up after about one second, record the timeout and return, and the
  * CUDA context stays usable.  Returns MOE_ERR_TIMEOUT when the wait ran out as
  * designed (the expected result), MOE_OK if it did not.  Synchronises
- * `stream`; ws needs moe_workspace_bytes(4096, 1, 8, 8) bytes. */
+ * `stream`; ws needs moe_workspace_bytes(4096, 1, 8, 8) bytes; the
+ * workspace's error words are cleared afterwards. */
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Kernel launches issued by this library on the calling thread since the
