@@ -67,6 +67,8 @@ def lib():
         L.oracle_fp8_rows.argtypes = [P, i64, i64, P, P]
         L.oracle_combine.argtypes = [P, P, P, i64, i32, i64, P]
         L.oracle_bias_update.argtypes = [P, i32, i64, f32, i32, P]
+        L.oracle_route_balanced.argtypes = [i64, i32, i32, f32, P, P]
+        L.oracle_bias_update_ema.argtypes = [P, i32, i64, f32, f32, P, P]
         _lib = L
     return _lib
 
@@ -252,9 +254,37 @@ def bias_update(counts, total, bias, u=0.001, mode=0) -> np.ndarray:
 
 
 def route(x, W, off, bias, fn, K, n_groups=1, topk_groups=1, group_topn=2, renorm=True,
-          scale=1.0):
-    """Gate -> scores -> selection, end to end on the CPU."""
+          scale=1.0, bias_in_logits=False):
+    """Gate -> scores -> selection, end to end on the CPU.
+
+    bias_in_logits: the bias joins the logits before the nonlinearity, as in
+    the DynamicEntropyMoERouter of "MoE Routing Entropy vs Expert
+    Saturation" ("Concrete Implementation": compensated_logits = raw_logits
+    + expert_biases), so it shapes the weights too and selection uses the
+    scores themselves; otherwise it only shifts the selection key."""
     h = logits(x, W, off)
+    if bias_in_logits and bias is not None:
+        h = h + np.asarray(bias, dtype=np.float64)[None, :]
     s = scores(h, fn)
-    idx, w = select(s, bias, K, n_groups, topk_groups, group_topn, renorm, scale)
+    idx, w = select(s, None if bias_in_logits else bias, K, n_groups, topk_groups, group_topn, renorm, scale)
     return h, s, idx, w
+
+
+def route_balanced(T, K, N, scale=1.0):
+    """Round-robin expert (t*K + k) mod N with equal weights scale/K: the
+    "forcible load balancing" upper bound of the MindIE load-balancer page."""
+    idx = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K), dtype=np.float32)
+    lib().oracle_route_balanced(T, K, N, float(scale), _p(idx), _p(w))
+    return idx, w
+
+
+def bias_update_ema(counts, total, bias, ema, u=0.001, alpha=0.9):
+    """Sign-rule bias step on an exponential moving average of the load
+    (hotdry aux-loss-free section: smoothed load statistics).  Returns
+    (new_bias, new_ema)."""
+    c = np.ascontiguousarray(counts, dtype=np.int64)
+    b = _f32(bias).copy()
+    e = _f32(ema).copy()
+    lib().oracle_bias_update_ema(_p(c), c.size, int(total), float(u), float(alpha), _p(e), _p(b))
+    return b, e

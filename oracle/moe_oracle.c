@@ -469,3 +469,39 @@ void oracle_bias_update(const int64_t* counts, int N, int64_t total, float u, in
         }
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * "Forcible load balancing" (MindIE expert_parallelism_load_balancer page:
+ * the top-k outputs are replaced by fake ones that balance the experts
+ * exactly, an upper bound for balance).  Reading: expert (t*K + k) mod N in
+ * round-robin order, equal weights route_scale / K.
+ * ------------------------------------------------------------------------- */
+void oracle_route_balanced(int64_t T, int K, int N, float route_scale, int32_t* idx, float* w) {
+    for (int64_t t = 0; t < T; ++t)
+        for (int k = 0; k < K; ++k) {
+            idx[t * K + k] = (int32_t)((t * K + k) % N);
+            w[t * K + k] = route_scale / (float)K;
+        }
+}
+
+/* ---------------------------------------------------------------------------
+ * Bias update on a smoothed load ("DeepSeek V4 MoE load balancing",
+ * aux-loss-free section: a moving average smooths the load statistics).
+ *   ema_e = fp32(fp32(alpha * ema_e) + fp32((1 - alpha) * c_e))
+ *   mean  = fp32(total / N)
+ *   b_e   = fp32(b_e - fp32(u * sign(ema_e - mean)))      (sign(0) = 0)
+ * every op a single fp32 rounding, in that order.
+ * ------------------------------------------------------------------------- */
+void oracle_bias_update_ema(const int64_t* counts, int N, int64_t total, float u, float alpha,
+                            float* ema, float* bias) {
+    const float mean = (float)((double)total / (double)N);
+    const float beta = 1.0f - alpha;
+    for (int e = 0; e < N; ++e) {
+        float a = alpha * ema[e];
+        float c = beta * (float)counts[e];
+        ema[e] = a + c;
+        float sgn = (float)((ema[e] > mean) - (ema[e] < mean));
+        float step = u * sgn;
+        bias[e] = bias[e] - step;
+    }
+}

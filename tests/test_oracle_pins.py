@@ -388,3 +388,64 @@ def test_bias_update_proportional_rule(orc):
     b = orc.bias_update(counts, 32, np.zeros(4, np.float32), 0.05, 1)
     q = np.float32(0.05) * np.float32(0.25)
     assert b.tolist() == [-q, q, 0.0, 0.0]
+
+
+# --------------------------------------------------------------------------------------
+# forcible balancing, bias in the logits, smoothed-load bias update
+# --------------------------------------------------------------------------------------
+def test_forcible_balance_is_exactly_balanced(orc):
+    for T, K, N in ((64, 1, 4), (1000, 8, 256), (513, 2, 8), (7, 3, 5)):
+        idx, w = orc.route_balanced(T, K, N, 2.5)
+        assert all(len(set(r)) == K for r in idx.tolist())        # distinct experts per token
+        c = orc.histogram(idx, N)
+        assert c.max() - c.min() <= 1 and c.sum() == T * K
+        np.testing.assert_allclose(w.astype(np.float64).sum(1), 2.5, rtol=1e-6)
+    # the page's four experts and 64 assignments: the balanced case of the worked example
+    idx, _ = orc.route_balanced(64, 1, 4)
+    st = orc.load_stats(orc.histogram(idx, 4))
+    assert st["imbalance"] == 1.0 and st["capacity_fixed"] == 64
+
+
+def test_bias_in_logits_softmax_shift_invariance(orc):
+    # a bias equal on every expert cancels in the softmax
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((30, 16)).astype(np.float32)
+    W = rng.standard_normal((8, 16)).astype(np.float32)
+    _, s0, i0, w0 = orc.route(x, W, None, None, 0, 2)
+    _, s1, i1, w1 = orc.route(x, W, None, np.full(8, 0.75, np.float32), 0, 2, bias_in_logits=True)
+    np.testing.assert_allclose(s1, s0, rtol=1e-6)
+    assert np.array_equal(i0, i1)
+
+
+def test_bias_in_logits_shapes_weights(orc):
+    # one token, equal logits: a logit bias of ln 3 on expert 2 makes it three
+    # times as likely as the others; selection-only bias would leave weights equal
+    x = np.zeros((1, 4), np.float32)
+    W = np.zeros((4, 4), np.float32)
+    b = np.array([0, 0, np.log(3.0), 0], np.float32)
+    _, s, idx, w = orc.route(x, W, None, b, 0, 2, bias_in_logits=True)
+    assert idx.tolist() == [[2, 0]]
+    assert w[0].tolist() == pytest.approx([0.75, 0.25], rel=1e-6)
+    _, s2, idx2, w2 = orc.route(x, W, None, b, 0, 2)
+    assert idx2.tolist() == [[2, 0]] and w2[0].tolist() == [0.5, 0.5]
+
+
+def test_bias_update_ema_reduces_to_sign_rule(orc):
+    counts = np.array([10, 6, 8, 8])
+    b0 = np.zeros(4, np.float32)
+    b, e = orc.bias_update_ema(counts, 32, b0, np.zeros(4, np.float32), 0.001, 0.0)
+    assert b.tolist() == orc.bias_update(counts, 32, b0, 0.001, 0).tolist()
+    assert e.tolist() == [10.0, 6.0, 8.0, 8.0]
+
+
+def test_bias_update_ema_smooths(orc):
+    # alpha = 0.5: the moving average moves halfway to the new load each step
+    counts = np.array([16, 0, 8, 8])
+    b, e = orc.bias_update_ema(counts, 32, np.zeros(4, np.float32), np.full(4, 8, np.float32), 0.001, 0.5)
+    assert e.tolist() == [12.0, 4.0, 8.0, 8.0]
+    assert b.tolist() == [-np.float32(0.001), np.float32(0.001), 0.0, 0.0]
+    # a load that stays constant: the average converges to it geometrically
+    e = np.zeros(4, np.float32)
+    for _ in range(40):
+        _, e = orc.bias_update_ema(counts, 32, np.zeros(4, np.float32), e, 0.001, 0.5)
+    np.testing.assert_allclose(e, counts, atol=1e-5)
