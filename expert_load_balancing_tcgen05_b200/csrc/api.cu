@@ -12,9 +12,13 @@ bool gate_tc_supported(int N);
 bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn);
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
-                           bool fused, float* scores, int32_t* idx, float* w, int32_t* err, cudaStream_t st);
-cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, int T, int d, int N,
-                             int fn, float* scores, cudaStream_t st);
+                           bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
+                           cudaStream_t st);
+cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, const float* logit_bias,
+                             int T, int d, int N, int fn, float* scores, cudaStream_t st);
+cudaError_t launch_bias_update_ema(const int32_t* counts, int N, int64_t total, float u, float alpha, float* ema,
+                                   float* bias, cudaStream_t st);
+cudaError_t launch_route_balanced(int64_t T, int K, int N, float scale, int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K, int n_groups,
                               int topk_groups, int group_topn, int renorm, float route_scale, int32_t* idx,
                               float* w, cudaStream_t st);
@@ -70,6 +74,7 @@ static moe_status check_route_cfg(const moe_route_cfg* c) {
     if (c == nullptr) return MOE_ERR_INVALID;
     if (c->T < 0 || c->N <= 0 || c->K <= 0 || c->K > c->N || c->K > 32) return MOE_ERR_INVALID;
     if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_INVALID;
+    if (c->bias_mode != 0 && c->bias_mode != 1) return MOE_ERR_INVALID;
     if (c->n_groups <= 0 || c->N % c->n_groups != 0 || c->n_groups > 32) return MOE_ERR_INVALID;
     const int gsize = c->N / c->n_groups;
     if (c->n_groups > 1) {
@@ -104,6 +109,9 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
     if (topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID;
     if (scores != nullptr && !aligned16(scores)) return MOE_ERR_INVALID;
     const int eff_topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
+    const bool bias_in_logits = c.bias_mode == 1;
+    if (bias_in_logits && x == nullptr) return MOE_ERR_INVALID;  // the bias needs the logits
+    const float* sel_bias = bias_in_logits ? nullptr : bias;
     const bool tensor_core = x != nullptr && c.in_dtype == MOE_BF16 && gate_tc_supported(c.N);
     const bool fused = tensor_core && gate_tc_can_fuse(c.N, c.K, c.score_fn, c.n_groups, c.group_topn) &&
                        (scores == nullptr || use_fused_select(c.T));
@@ -120,16 +128,17 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
         if (tensor_core) {
             if (c.d % 8 != 0 || !aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID;
             e = launch_gate_tc(x, w_gate, logit_offset, bias, c.T, c.d, c.N, c.K, c.score_fn, c.n_groups,
-                               eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, fused, scores,
-                               topk_idx, topk_w, &hdr->gate_err, st);
+                               eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, fused,
+                               bias_in_logits, scores, topk_idx, topk_w, &hdr->gate_err, st);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
             if (fused) return MOE_OK;
         } else {
-            e = launch_gate_simt(x, w_gate, c.in_dtype, logit_offset, c.T, c.d, c.N, c.score_fn, scores, st);
+            e = launch_gate_simt(x, w_gate, c.in_dtype, logit_offset, bias_in_logits ? bias : nullptr, c.T, c.d, c.N,
+                                 c.score_fn, scores, st);
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    return cuda_status(launch_route_topk(scores, bias, c.T, c.N, c.K, c.n_groups, eff_topk_groups,
+    return cuda_status(launch_route_topk(scores, sel_bias, c.T, c.N, c.K, c.n_groups, eff_topk_groups,
                                          c.group_topn, c.renorm ? 1 : 0, c.route_scale, topk_idx, topk_w, st));
 }
 
@@ -147,6 +156,24 @@ moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t
     if (ws_bytes < moe_workspace_bytes(T, K, N, n_slots)) return MOE_ERR_INVALID;
     return cuda_status(launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets, rank,
                                          scores, score_fn, stats, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale, int32_t* topk_idx,
+                              float* topk_w, moe_stream_t stream) {
+    if (T < 0 || K <= 0 || N <= 0 || K > N || T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
+    if (T > 0 && (topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID;
+    if (T == 0) return MOE_OK;
+    return cuda_status(launch_route_balanced(T, K, N, route_scale, topk_idx, topk_w,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_bias_update_ema(const int32_t* counts, int32_t N, int64_t total_assignments, float u, float alpha,
+                               float* load_ema, float* bias, moe_stream_t stream) {
+    if (counts == nullptr || load_ema == nullptr || bias == nullptr || N <= 0 || total_assignments <= 0 ||
+        !(alpha >= 0.f && alpha < 1.f))
+        return MOE_ERR_INVALID;
+    return cuda_status(launch_bias_update_ema(counts, N, total_assignments, u, alpha, load_ema, bias,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_replica_plan(const int32_t* counts, int32_t N, int32_t n_replicas, int32_t* replica_slot,

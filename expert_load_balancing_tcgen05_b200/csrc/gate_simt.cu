@@ -1,7 +1,8 @@
 // Gate logits and scores on CUDA cores, for fp32 inputs (and for bf16
 // expert counts the tensor-core kernel has no tile for).
 //
-// h[t,e] = sum_j x[t,j] * W[e,j] + off[e] ("MoE Routing Entropy vs Expert
+// h[t,e] = sum_j x[t,j] * W[e,j] + off[e] (+ b[e] when the bias joins the
+// logits) ("MoE Routing Entropy vs Expert
 // Saturation", section "The Mathematics": h = x . W_g with the nn.Linear gate
 // of section "Concrete Implementation"); then softmax over the experts (same
 // section) or sigmoid ("DeepSeek V4 MoE load balancing", token routing).
@@ -26,7 +27,8 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return _
 
 template <typename TIn>
 __global__ void __launch_bounds__(256) gate_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ W,
-                                                        const float* __restrict__ off, int T, int d, int N,
+                                                        const float* __restrict__ off,
+                                                        const float* __restrict__ logit_bias, int T, int d, int N,
                                                         int fn, float* __restrict__ scores) {
     const int lane = threadIdx.x & 31;
     const int wpb = blockDim.x >> 5;
@@ -42,6 +44,7 @@ __global__ void __launch_bounds__(256) gate_simt_kernel(const TIn* __restrict__ 
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
             if (off != nullptr) acc += off[e];
+            if (logit_bias != nullptr) acc += logit_bias[e];
             // lane e%32 keeps h_e in register slot e/32 (unrolled select keeps h in registers)
 #pragma unroll
             for (int i = 0; i < MAX_N / 32; ++i)
@@ -78,19 +81,19 @@ __global__ void __launch_bounds__(256) gate_simt_kernel(const TIn* __restrict__ 
     }
 }
 
-cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, int T, int d, int N,
-                             int fn, float* scores, cudaStream_t st) {
+cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, const float* logit_bias,
+                             int T, int d, int N, int fn, float* scores, cudaStream_t st) {
     long long blocks = ((long long)T + 7) / 8;
     const long long cap = (long long)moe_host::sm_count() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (dtype == MOE_F32)
         gate_simt_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
-            static_cast<const float*>(x), static_cast<const float*>(W), off, T, d, N, fn, scores);
+            static_cast<const float*>(x), static_cast<const float*>(W), off, logit_bias, T, d, N, fn, scores);
     else
         gate_simt_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W), off, T, d, N, fn,
-            scores);
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W), off, logit_bias, T, d, N,
+            fn, scores);
     moe_host::note_launch();
     return cudaGetLastError();
 }

@@ -167,6 +167,7 @@ struct Epi {
     int32_t* idx;       // [T, K]
     float* w;           // [T, K]
     int T, fn, K, n_groups, topk_groups, group_topn, renorm, fused;
+    int bias_in_logits;  // the bias joins the logit offset; the selection key is the score itself
     float scale;
 };
 
@@ -351,8 +352,10 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     for (int i = threadIdx.x; i < BN; i += blockDim.x) {
-        off_s[i] = p.off != nullptr ? p.off[i] : 0.f;
-        bias_s[i] = p.bias != nullptr ? p.bias[i] : 0.f;
+        const float o = p.off != nullptr ? p.off[i] : 0.f;
+        const float b = p.bias != nullptr ? p.bias[i] : 0.f;
+        off_s[i] = p.bias_in_logits ? __fadd_rn(o, b) : o;
+        bias_s[i] = p.bias_in_logits ? 0.f : b;
     }
     fence_before();
     __syncthreads();
@@ -570,8 +573,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     for (int i = threadIdx.x; i < BN; i += blockDim.x) {
-        off_s[i] = p.off != nullptr ? p.off[i] : 0.f;
-        bias_s[i] = p.bias != nullptr ? p.bias[i] : 0.f;
+        const float o = p.off != nullptr ? p.off[i] : 0.f;
+        const float b = p.bias != nullptr ? p.bias[i] : 0.f;
+        off_s[i] = p.bias_in_logits ? __fadd_rn(o, b) : o;
+        bias_s[i] = p.bias_in_logits ? 0.f : b;
     }
     fence_before();
     cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
@@ -752,8 +757,10 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
 
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
-                           bool fused, float* scores, int32_t* idx, float* w, int32_t* err, cudaStream_t st) {
+                           bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
+                           cudaStream_t st) {
     tc::Epi p;
+    p.bias_in_logits = bias_in_logits ? 1 : 0;
     p.off = off; p.bias = bias; p.scores = scores; p.idx = idx; p.w = w;
     p.T = T; p.fn = fn; p.K = K; p.n_groups = n_groups; p.topk_groups = topk_groups; p.group_topn = group_topn;
     p.renorm = renorm; p.fused = fused ? 1 : 0; p.scale = scale;

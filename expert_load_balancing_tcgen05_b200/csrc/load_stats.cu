@@ -459,6 +459,30 @@ __global__ void __launch_bounds__(1024) bias_update_kernel(const int32_t* __rest
     }
 }
 
+// smoothed-load bias step: ema = fp32(fp32(alpha*ema) + fp32((1-alpha)*c)),
+// b -= fp32(u * sign(ema - fp32(total/N)))
+__global__ void __launch_bounds__(1024) bias_update_ema_kernel(const int32_t* __restrict__ counts, int N,
+                                                               int64_t total, float u, float alpha,
+                                                               float* __restrict__ ema, float* __restrict__ bias) {
+    const float mean = (float)((double)total / (double)N);
+    const float beta = __fsub_rn(1.f, alpha);
+    for (int e = threadIdx.x; e < N; e += blockDim.x) {
+        const float v = __fadd_rn(__fmul_rn(alpha, ema[e]), __fmul_rn(beta, (float)counts[e]));
+        ema[e] = v;
+        const float sgn = (float)((v > mean) - (v < mean));
+        bias[e] = __fsub_rn(bias[e], __fmul_rn(u, sgn));
+    }
+}
+
+// forcible balancing: expert (t*K + k) mod N, weight scale / K
+__global__ void __launch_bounds__(256) route_balanced_kernel(int64_t A, int K, int N, float w,
+                                                             int32_t* __restrict__ idx, float* __restrict__ wout) {
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A; a += (int64_t)gridDim.x * blockDim.x) {
+        idx[a] = (int32_t)(a % N);
+        wout[a] = w;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
@@ -532,6 +556,24 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
 
 cudaError_t launch_replica_plan(const int32_t* counts, int N, int R, int32_t* replica_slot, cudaStream_t st) {
     replica_plan_kernel<<<1, 1024, sizeof(int32_t) * (size_t)N, st>>>(counts, N, R, replica_slot);
+    moe_host::note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update_ema(const int32_t* counts, int N, int64_t total, float u, float alpha, float* ema,
+                                   float* bias, cudaStream_t st) {
+    bias_update_ema_kernel<<<1, 1024, 0, st>>>(counts, N, total, u, alpha, ema, bias);
+    moe_host::note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_balanced(int64_t T, int K, int N, float scale, int32_t* idx, float* w, cudaStream_t st) {
+    const int64_t A = T * K;
+    long long blocks = (A + 255) / 256;
+    const long long cap = (long long)moe_host::sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    route_balanced_kernel<<<(unsigned)blocks, 256, 0, st>>>(A, K, N, scale / (float)K, idx, w);
     moe_host::note_launch();
     return cudaGetLastError();
 }

@@ -28,14 +28,15 @@ MOE_F32, MOE_BF16 = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
-           "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout")
+           "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout", "moe_route_balanced",
+           "moe_bias_update_ema")
 
 
 class RouteCfg(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("score_fn", ctypes.c_int32), ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
                 ("group_topn", ctypes.c_int32), ("renorm", ctypes.c_int32), ("route_scale", ctypes.c_float),
-                ("in_dtype", ctypes.c_int32)]
+                ("in_dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32)]
 
 
 class Stats(ctypes.Structure):
@@ -130,6 +131,22 @@ def moe_load_stats_noalloc(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, c
                                        _ptr(stats), _stream(stream)), "moe_load_stats_noalloc")
 
 
+_lib.moe_route_balanced.argtypes = [_I64, _I32, _I32, _F32, _P, _P, _P]
+_lib.moe_route_balanced.restype = _I32
+_lib.moe_bias_update_ema.argtypes = [_P, _I32, _I64, _F32, _F32, _P, _P, _P]
+_lib.moe_bias_update_ema.restype = _I32
+
+
+def moe_route_balanced(T, K, N, route_scale, topk_idx, topk_w, stream=None):
+    _check(_lib.moe_route_balanced(T, K, N, float(route_scale), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+           "moe_route_balanced")
+
+
+def moe_bias_update_ema(counts, N, total_assignments, u, alpha, load_ema, bias, stream=None):
+    _check(_lib.moe_bias_update_ema(_ptr(counts), N, total_assignments, float(u), float(alpha), _ptr(load_ema),
+                                    _ptr(bias), _stream(stream)), "moe_bias_update_ema")
+
+
 def moe_replica_plan(counts, N, n_replicas, replica_slot, stream=None):
     _check(_lib.moe_replica_plan(_ptr(counts), N, n_replicas, _ptr(replica_slot), _stream(stream)),
            "moe_replica_plan")
@@ -175,9 +192,9 @@ def moe_version() -> str:
 # small conveniences (allocation of caller-owned buffers, decoding the stats struct)
 # --------------------------------------------------------------------------------------
 def route_cfg(T, d, N, K, score_fn, n_groups=1, topk_groups=1, group_topn=2, renorm=True, route_scale=1.0,
-              in_dtype=MOE_BF16) -> RouteCfg:
+              in_dtype=MOE_BF16, bias_in_logits=False) -> RouteCfg:
     return RouteCfg(T, d, N, K, score_fn, n_groups, topk_groups, group_topn, 1 if renorm else 0,
-                    float(route_scale), in_dtype)
+                    float(route_scale), in_dtype, 1 if bias_in_logits else 0)
 
 
 def empty_stats(device="cuda") -> torch.Tensor:

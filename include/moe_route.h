@@ -66,6 +66,10 @@ typedef struct {
     int32_t renorm;       /* 1: weights = s_k / sum of chosen s; 0: weights = s_k */
     float route_scale;    /* weights are multiplied by this (2.5 for V3 routing) */
     int32_t in_dtype;     /* moe_dtype of x and w_gate */
+    int32_t bias_mode;    /* 0: bias only in the selection key (aux-loss-free routing);
+                             1: bias added to the logits before the nonlinearity, so it
+                                also shapes the weights ([ENT] "Concrete Implementation":
+                                compensated_logits = raw_logits + expert_biases); needs x */
 } moe_route_cfg;
 
 /* Load statistics of one histogram, written to device memory.
@@ -134,6 +138,17 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
                      moe_stream_t stream);
 
 /*
+ * moe_route_balanced -- "forcible load balancing": the top-K output replaced
+ * by an exactly balanced one, an upper bound for balance experiments
+ * (MindIE expert_parallelism_load_balancer page, forcible load balancing).
+ *   topk_idx[t,k] = (t*K + k) mod N,  topk_w[t,k] = route_scale / K
+ * Every expert gets T*K/N assignments (+-1); a token's K experts are
+ * distinct (K <= N).
+ */
+moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale, int32_t* topk_idx,
+                              float* topk_w, moe_stream_t stream);
+
+/*
  * moe_load_stats -- load histogram, expert offsets, stable in-expert ranks
  * and load statistics.
  *
@@ -184,6 +199,19 @@ moe_status moe_replica_plan(const int32_t* counts, int32_t N, int32_t n_replicas
  */
 moe_status moe_bias_update(const int32_t* counts, int32_t N, int64_t total_assignments,
                            float u, int32_t mode, float* bias, moe_stream_t stream);
+
+/*
+ * moe_bias_update_ema -- the sign-rule bias step on a smoothed load ([HD]
+ * "Auxiliary-loss-free load balancing": a moving average smooths the load
+ * statistics before the bias is adjusted).  In place on load_ema [N] and
+ * bias [N] (fp32, caller-owned state; start load_ema at 0 or at a first
+ * histogram):
+ *   load_ema_e = fp32(fp32(alpha * load_ema_e) + fp32((1 - alpha) * c_e))
+ *   b_e        = fp32(b_e - fp32(u * sign(load_ema_e - fp32(total / N))))
+ * alpha in [0, 1); alpha = 0 is the plain sign rule on this step's counts.
+ */
+moe_status moe_bias_update_ema(const int32_t* counts, int32_t N, int64_t total_assignments, float u,
+                               float alpha, float* load_ema, float* bias, moe_stream_t stream);
 
 /*
  * moe_dispatch -- scatter token rows into the expert-contiguous buffer

@@ -84,6 +84,28 @@ def test_route_rejects_null_outputs_and_workspace(moe):
     assert L.moe_route(ctypes.byref(cfg), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, 16, None) == 1
 
 
+def test_route_bias_mode_validation(moe):
+    L = moe._lib
+    # unknown mode; the bias in the logits needs the gate input
+    assert L.moe_route(ctypes.byref(_cfg(moe, bias_mode=2)), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE,
+                       1 << 20, None) == 1
+    assert L.moe_route(ctypes.byref(_cfg(moe, bias_mode=1)), None, None, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                       1 << 20, None) == 1
+
+
+def test_balanced_and_ema_reject_bad_arguments(moe):
+    L = moe._lib
+    assert L.moe_route_balanced(-1, 8, 256, 1.0, FAKE, FAKE, None) == 1
+    assert L.moe_route_balanced(16, 0, 256, 1.0, FAKE, FAKE, None) == 1
+    assert L.moe_route_balanced(16, 300, 256, 1.0, FAKE, FAKE, None) == 1
+    assert L.moe_route_balanced(16, 8, 256, 1.0, None, FAKE, None) == 1
+    assert L.moe_route_balanced(0, 8, 256, 1.0, None, None, None) == 0  # empty batch: nothing to write
+    assert L.moe_bias_update_ema(FAKE, 256, 100, 0.001, 1.0, FAKE, FAKE, None) == 1
+    assert L.moe_bias_update_ema(FAKE, 256, 100, 0.001, -0.5, FAKE, FAKE, None) == 1
+    assert L.moe_bias_update_ema(FAKE, 256, 0, 0.001, 0.9, FAKE, FAKE, None) == 1
+    assert L.moe_bias_update_ema(FAKE, 256, 100, 0.001, 0.9, None, FAKE, None) == 1
+
+
 def test_load_stats_rejects_bad_arguments(moe):
     L = moe._lib
     ws = 1 << 24
