@@ -69,6 +69,8 @@ def lib():
         L.oracle_bias_update.argtypes = [P, i32, i64, f32, i32, P]
         L.oracle_route_balanced.argtypes = [i64, i32, i32, f32, P, P]
         L.oracle_bias_update_ema.argtypes = [P, i32, i64, f32, f32, P, P]
+        L.oracle_route_capacity.argtypes = [P, P, i64, i32, i32, i32, i32, i32, i32, f32, i64, P, P, P]
+        L.oracle_route_capacity.restype = i32
         _lib = L
     return _lib
 
@@ -288,3 +290,30 @@ def bias_update_ema(counts, total, bias, ema, u=0.001, alpha=0.9):
     e = _f32(ema).copy()
     lib().oracle_bias_update_ema(_p(c), c.size, int(total), float(u), float(alpha), _p(e), _p(b))
     return b, e
+
+
+def capacity_limit(T, K, N, factor_quarters=5):
+    """ceil(1.25 * T*K/N) in integers: the per-expert token capacity of the
+    "Production Testing" section of the entropy page."""
+    return (factor_quarters * T * K + 4 * N - 1) // (4 * N)
+
+
+def route_capacity(s, bias, K, n_groups=1, topk_groups=1, group_topn=2, renorm=True, scale=1.0,
+                   capacity=None):
+    """Capacity-limited selection on fp32 scores: primaries accepted in flat
+    (t, k) order up to the capacity, each token's overflowed slots moved to
+    its next ranked candidates, the rest dropped (idx -1, weight 0).
+    Returns (idx, w, info) with info = {capacity, overflow, rerouted, dropped}."""
+    s = _f32(s)
+    T, N = s.shape
+    C = capacity_limit(T, K, N) if capacity is None else int(capacity)
+    b = _f32(bias) if bias is not None else None
+    idx = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K), dtype=np.float32)
+    info = np.zeros(3, dtype=np.int64)
+    rc = lib().oracle_route_capacity(_p(s), _p(b) if b is not None else None, T, N, K, n_groups,
+                                     topk_groups, group_topn, 1 if renorm else 0, float(scale), C,
+                                     _p(idx), _p(w), _p(info))
+    if rc != 0:
+        raise ValueError("oracle_route_capacity: invalid configuration")
+    return idx, w, dict(capacity=C, overflow=int(info[0]), rerouted=int(info[1]), dropped=int(info[2]))

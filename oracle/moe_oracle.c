@@ -201,12 +201,15 @@ int oracle_select(const float* s, const float* bias, int64_t T, int N, int K,
 
 /* ---------------------------------------------------------------------------
  * Load histogram: c_e = #{(t,k) : slot(t,k) = e}  ([ENT] "Concrete
- * Implementation", bincount of the selected experts).
+ * Implementation", bincount of the selected experts).  A negative slot is an
+ * assignment dropped by the capacity limit ([ENT] "Production Testing") and
+ * counts nowhere.
  * ------------------------------------------------------------------------- */
 int oracle_histogram(const int32_t* slot, int64_t A, int n_slots, int64_t* counts) {
     for (int e = 0; e < n_slots; ++e) counts[e] = 0;
     for (int64_t a = 0; a < A; ++a) {
-        if (slot[a] < 0 || slot[a] >= n_slots) return -1;
+        if (slot[a] < 0) continue;
+        if (slot[a] >= n_slots) return -1;
         counts[slot[a]] += 1;
     }
     return 0;
@@ -311,7 +314,7 @@ void oracle_apply_replicas(const int32_t* idx, int64_t T, int K,
     for (int64_t t = 0; t < T; ++t)
         for (int k = 0; k < K; ++k) {
             int32_t e = idx[t * K + k];
-            int32_t r = replica_slot ? replica_slot[e] : -1;
+            int32_t r = (replica_slot && e >= 0) ? replica_slot[e] : -1;
             slot[t * K + k] = (r >= 0 && (t & 1)) ? r : e;
         }
 }
@@ -321,7 +324,8 @@ void oracle_apply_replicas(const int32_t* idx, int64_t T, int K,
  * experts, combine brings the results back).  offsets = exclusive prefix of
  * counts (n_slots + 1 entries); walking the flat assignments a = t*K + k in
  * ascending order, pos[a] = offsets[e] + rank[a] with rank[a] the number of
- * earlier assignments to the same slot; row_src[pos[a]] = t.
+ * earlier assignments to the same slot; row_src[pos[a]] = t.  A dropped
+ * assignment (negative slot) gets rank = pos = -1 and no row.
  * ------------------------------------------------------------------------- */
 void oracle_positions(const int32_t* slot, int64_t T, int K, const int64_t* counts,
                       int n_slots, int64_t* offsets, int64_t* pos, int64_t* rank,
@@ -331,6 +335,7 @@ void oracle_positions(const int32_t* slot, int64_t T, int K, const int64_t* coun
     int64_t* seen = (int64_t*)calloc((size_t)n_slots, sizeof(int64_t));
     for (int64_t a = 0; a < T * K; ++a) {
         int32_t e = slot[a];
+        if (e < 0) { rank[a] = -1; pos[a] = -1; continue; }
         rank[a] = seen[e];
         pos[a] = offsets[e] + seen[e];
         seen[e] += 1;
@@ -339,12 +344,13 @@ void oracle_positions(const int32_t* slot, int64_t T, int K, const int64_t* coun
     free(seen);
 }
 
-/* rows[pos[t,k]] = x[t]: a byte copy of each token row, K times. */
+/* rows[pos[t,k]] = x[t]: a byte copy of each token row, K times (dropped
+ * assignments, pos < 0, copy nothing). */
 void oracle_dispatch_rows(const uint8_t* x, int64_t T, int64_t row_bytes, int K,
                           const int64_t* pos, uint8_t* rows) {
     for (int64_t t = 0; t < T; ++t)
         for (int k = 0; k < K; ++k)
-            memcpy(rows + pos[t * K + k] * row_bytes, x + t * row_bytes, (size_t)row_bytes);
+            if (pos[t * K + k] >= 0) memcpy(rows + pos[t * K + k] * row_bytes, x + t * row_bytes, (size_t)row_bytes);
 }
 
 /* ---------------------------------------------------------------------------
@@ -426,7 +432,8 @@ void oracle_fp8_rows(const float* rows, int64_t R, int64_t d, uint8_t* q, float*
 /* ---------------------------------------------------------------------------
  * Combine ([HD] "Token routing": expert outputs are summed weighted by their
  * affinity; "DeepEP": combine returns them to the token's place):
- * out[t] = sum_k w[t,k] * y[pos[t,k]], in double, k order.
+ * out[t] = sum_k w[t,k] * y[pos[t,k]], in double, k order; dropped
+ * assignments (pos < 0) contribute nothing.
  * ------------------------------------------------------------------------- */
 void oracle_combine(const float* y, const int64_t* pos, const float* w, int64_t T,
                     int K, int64_t d, double* out) {
@@ -436,7 +443,7 @@ void oracle_combine(const float* y, const int64_t* pos, const float* w, int64_t 
         for (int64_t j = 0; j < d; ++j) {
             double acc = 0.0;
             for (int k = 0; k < K; ++k)
-                acc += (double)w[t * K + k] * (double)y[pos[t * K + k] * d + j];
+                if (pos[t * K + k] >= 0) acc += (double)w[t * K + k] * (double)y[pos[t * K + k] * d + j];
             out[t * d + j] = acc;
         }
 }
@@ -504,4 +511,139 @@ void oracle_bias_update_ema(const int64_t* counts, int N, int64_t total, float u
         float step = u * sgn;
         bias[e] = bias[e] - step;
     }
+}
+
+/* ---------------------------------------------------------------------------
+ * Capacity-limited routing ([ENT] "Production Testing": a hard token capacity
+ * per expert, 1.25 * T*K/N, with the excess routed to secondary candidate
+ * experts by the bias-adjusted ranking).
+ *  1. Candidates of token t: the experts of its kept groups (selection step
+ *     2), ranked by (key desc, index asc) with key = fp32(s + b); the first K
+ *     are the selection's choice, in its order.
+ *  2. Primary pass, flat order a = t*K + k: an assignment is accepted while
+ *     its expert has accepted fewer than C; otherwise it overflows.
+ *  3. Reroute pass: token t's j-th overflowed slot (counting in k order) takes
+ *     candidate K + j, if the token has that many.  In flat order again, a
+ *     rerouted assignment is accepted while its expert holds fewer than C in
+ *     all (primaries and earlier reroutes).  Anything else is dropped:
+ *     idx -1, weight 0.  One reroute round; a second overflow is a drop.
+ *  4. Weights from the unbiased scores of the token's final experts:
+ *     renorm ? s / (sum over its kept slots in k order) : s, times
+ *     route_scale, each op rounded to fp32 (a token with every slot dropped
+ *     gets zero weights).
+ * info[0] = overflowed primaries, info[1] = accepted reroutes, info[2] =
+ * dropped assignments.  Returns 0, or -1 on an invalid configuration.
+ * ------------------------------------------------------------------------- */
+typedef struct { float key; int e; } cap_cand;
+
+static int cap_cand_cmp(const void* a, const void* b) {
+    const cap_cand* x = (const cap_cand*)a;
+    const cap_cand* y = (const cap_cand*)b;
+    if (beats(x->key, x->e, y->key, y->e)) return -1;
+    if (beats(y->key, y->e, x->key, x->e)) return 1;
+    return 0;
+}
+
+int oracle_route_capacity(const float* s, const float* bias, int64_t T, int N, int K,
+                          int n_groups, int topk_groups, int group_topn, int renorm,
+                          float route_scale, int64_t C, int32_t* idx, float* w, int64_t* info) {
+    if (N <= 0 || K <= 0 || K > N || n_groups <= 0 || N % n_groups || C < 0) return -1;
+    const int gsize = N / n_groups;
+    if (n_groups > 1 && (topk_groups <= 0 || topk_groups > n_groups ||
+                         topk_groups * gsize < K || group_topn <= 0 || group_topn > gsize))
+        return -1;
+    /* ranked candidates: second[t*K + j] = candidate K + j, or -1 */
+    int32_t* second = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T * K + 1));
+    int64_t* used = (int64_t*)calloc((size_t)N, sizeof(int64_t));
+    int32_t* fin = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T * K + 1));
+    if (!second || !used || !fin) { free(second); free(used); free(fin); return -1; }
+    int64_t t;
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (t = 0; t < T; ++t) {
+        float* key = (float*)malloc(sizeof(float) * (size_t)N);
+        float* gs = (float*)malloc(sizeof(float) * (size_t)n_groups);
+        float* tmp = (float*)malloc(sizeof(float) * (size_t)gsize);
+        cap_cand* cand = (cap_cand*)malloc(sizeof(cap_cand) * (size_t)N);
+        if (!key || !gs || !tmp || !cand) { bad |= 1; goto next; }
+        for (int e = 0; e < N; ++e) key[e] = s[t * N + e] + (bias ? bias[e] : 0.0f);
+        int nc = 0;
+        for (int g = 0; g < n_groups; ++g) {
+            int keep = 1;
+            if (n_groups > 1) {
+                /* group scores as in the selection, then this group's rank */
+                for (int h2 = 0; h2 < n_groups; ++h2) {
+                    for (int i = 0; i < gsize; ++i) tmp[i] = key[h2 * gsize + i];
+                    float sum = 0.0f;
+                    for (int r = 0; r < group_topn; ++r) {
+                        int best = 0;
+                        for (int i = 1; i < gsize; ++i) if (tmp[i] > tmp[best]) best = i;
+                        sum = (r == 0) ? tmp[best] : sum + tmp[best];
+                        tmp[best] = -INFINITY;
+                    }
+                    gs[h2] = sum;
+                }
+                int rank = 0;
+                for (int h2 = 0; h2 < n_groups; ++h2)
+                    if (h2 != g && beats(gs[h2], h2, gs[g], g)) ++rank;
+                keep = rank < topk_groups;
+            }
+            if (keep)
+                for (int i = 0; i < gsize; ++i) {
+                    cand[nc].key = key[g * gsize + i];
+                    cand[nc].e = g * gsize + i;
+                    ++nc;
+                }
+        }
+        qsort(cand, (size_t)nc, sizeof(cap_cand), cap_cand_cmp);
+        for (int k = 0; k < K; ++k) {
+            idx[t * K + k] = cand[k].e;
+            second[t * K + k] = (K + k < nc) ? cand[K + k].e : -1;
+        }
+    next:
+        free(key); free(gs); free(tmp); free(cand);
+    }
+    if (bad) { free(second); free(used); free(fin); return -1; }
+
+    int64_t n_over = 0, n_rer = 0, n_drop = 0;
+    /* 2. primary pass */
+    for (int64_t a = 0; a < T * K; ++a) {
+        const int32_t e = idx[a];
+        if (used[e] < C) { used[e] += 1; fin[a] = e; }
+        else { fin[a] = -2; ++n_over; } /* -2: overflowed, to reroute */
+    }
+    /* 3. reroute pass */
+    for (int64_t tt = 0; tt < T; ++tt) {
+        int j = 0;
+        for (int k = 0; k < K; ++k) {
+            const int64_t a = tt * K + k;
+            if (fin[a] != -2) continue;
+            const int32_t e2 = second[tt * K + j];
+            ++j;
+            if (e2 >= 0 && used[e2] < C) { used[e2] += 1; fin[a] = e2; ++n_rer; }
+            else { fin[a] = -1; ++n_drop; }
+        }
+    }
+    /* 4. weights */
+    for (int64_t tt = 0; tt < T; ++tt) {
+        float ssum = 0.0f;
+        int first = 1;
+        for (int k = 0; k < K; ++k) {
+            const int32_t e = fin[tt * K + k];
+            if (e < 0) continue;
+            ssum = first ? s[tt * N + e] : ssum + s[tt * N + e];
+            first = 0;
+        }
+        for (int k = 0; k < K; ++k) {
+            const int32_t e = fin[tt * K + k];
+            idx[tt * K + k] = e;
+            if (e < 0) { w[tt * K + k] = 0.0f; continue; }
+            const float sk = s[tt * N + e];
+            const float v = renorm ? sk / ssum : sk;
+            w[tt * K + k] = v * route_scale;
+        }
+    }
+    info[0] = n_over; info[1] = n_rer; info[2] = n_drop;
+    free(second); free(used); free(fin);
+    return 0;
 }

@@ -449,3 +449,123 @@ def test_bias_update_ema_smooths(orc):
     for _ in range(40):
         _, e = orc.bias_update_ema(counts, 32, np.zeros(4, np.float32), e, 0.001, 0.5)
     np.testing.assert_allclose(e, counts, atol=1e-5)
+
+
+# --- dropped assignments and capacity-limited routing ("Production Testing") ---
+
+def test_dropped_assignments_take_no_slot(orc):
+    # hand example: token 1's second slot is dropped (-1)
+    slot = np.array([[0, 1], [1, -1], [0, 1]], np.int32)
+    counts, offsets, pos, rank, row_src = orc.positions(slot, 2)
+    assert counts.tolist() == [2, 3]
+    assert offsets.tolist() == [0, 2, 5]
+    assert pos.tolist() == [[0, 2], [3, -1], [1, 4]]
+    assert rank.tolist() == [[0, 0], [1, -1], [1, 2]]
+    assert row_src[:5].tolist() == [0, 2, 0, 1, 2]
+    x = np.arange(6, dtype=np.float32).reshape(3, 2)
+    rows = orc.dispatch_rows(x, pos)
+    assert rows[:5].tolist() == [[0, 1], [4, 5], [0, 1], [2, 3], [4, 5]]
+    # combine skips the dropped slot even with a nonzero weight
+    w = np.array([[1, 1], [1, 7], [1, 1]], np.float32)
+    out = orc.combine(rows[:5], pos, w)
+    assert out.tolist() == [[0, 2], [2, 3], [8, 10]]
+    assert orc.histogram(slot, 2).tolist() == [2, 3]
+    with pytest.raises(ValueError):
+        orc.histogram(np.array([[2]], np.int32), 2)
+
+
+def test_capacity_limit_value(orc):
+    # 1.25 * T*K/N, rounded up: 1.25 * 16384*8/256 = 640 exactly; 1.875 -> 2
+    assert orc.capacity_limit(16384, 8, 256) == 640
+    assert orc.capacity_limit(6, 1, 4) == 2
+    assert orc.capacity_limit(3, 2, 4) == 2
+    assert orc.capacity_limit(7, 1, 4) == 3  # 2.1875
+
+
+def test_capacity_hand_example_single_slot(orc):
+    # six tokens all preferring expert 0 then 1; capacity 2: tokens 0, 1 keep
+    # expert 0, tokens 2, 3 move to expert 1, tokens 4, 5 find it full
+    s = np.tile(np.array([0.9, 0.5, 0.3, 0.1], np.float32), (6, 1))
+    idx, w, info = orc.route_capacity(s, None, 1)
+    assert info == dict(capacity=2, overflow=4, rerouted=2, dropped=2)
+    assert idx[:, 0].tolist() == [0, 0, 1, 1, -1, -1]
+    assert w[:, 0].tolist() == [1, 1, 1, 1, 0, 0]
+
+
+def test_capacity_hand_example_two_slots(orc):
+    # both slots of token 2 overflow; its 1st overflow takes candidate 3 (rank
+    # K+0), the 2nd candidate 4 (rank K+1); weights renormalise over them
+    s = np.array([[0.9, 0.8, 0.2, 0.1], [0.9, 0.8, 0.2, 0.1], [0.9, 0.8, 0.3, 0.2]], np.float32)
+    idx, w, info = orc.route_capacity(s, None, 2, scale=2.0)
+    assert info == dict(capacity=2, overflow=2, rerouted=2, dropped=0)
+    assert idx.tolist() == [[0, 1], [0, 1], [2, 3]]
+    den = np.float32(0.3) + np.float32(0.2)
+    assert w[2].tolist() == [np.float32(np.float32(0.3) / den) * np.float32(2.0),
+                             np.float32(np.float32(0.2) / den) * np.float32(2.0)]
+
+
+def test_capacity_primaries_before_reroutes(orc):
+    # the primary pass finishes before any reroute: token 2's primary on
+    # expert 1 wins over token 1's reroute there, which is dropped
+    s = np.array([[0.9, 0.5, 0.1], [0.9, 0.5, 0.1], [0.1, 0.9, 0.5]], np.float32)
+    idx, w, info = orc.route_capacity(s, None, 1, capacity=1)
+    assert idx[:, 0].tolist() == [0, -1, 1]
+    assert info == dict(capacity=1, overflow=1, rerouted=0, dropped=1)
+
+
+def test_capacity_unbounded_is_plain_selection(orc):
+    g = np.random.default_rng(8)
+    s = g.random((300, 64)).astype(np.float32)
+    b = g.uniform(-0.05, 0.05, 64).astype(np.float32)
+    for kw in (dict(), dict(n_groups=8, topk_groups=3, group_topn=2)):
+        ri, rw = orc.select(s, b, 6, renorm=True, scale=2.5, **kw)
+        ci, cw, info = orc.route_capacity(s, b, 6, renorm=True, scale=2.5, capacity=300 * 6, **kw)
+        assert np.array_equal(ci, ri) and np.array_equal(cw, rw)
+        assert info["overflow"] == 0
+
+
+def test_capacity_zero_drops_everything(orc):
+    s = np.random.default_rng(1).random((10, 16)).astype(np.float32)
+    idx, w, info = orc.route_capacity(s, None, 4, capacity=0)
+    assert (idx == -1).all() and (w == 0).all()
+    assert info == dict(capacity=0, overflow=40, rerouted=0, dropped=40)
+
+
+@pytest.mark.parametrize("grouped", [False, True])
+def test_capacity_invariants(orc, grouped):
+    """Against the pinned selection and positions: primaries kept exactly when
+    their stable in-expert rank is below C; the j-th overflowed slot of a
+    token moves to its (K+j)-th ranked candidate (selection with 2K) or is
+    dropped; no expert exceeds C; kept weights renormalise to the scale."""
+    g = np.random.default_rng(21)
+    T, N, K = 700, 64, 4
+    kw = dict(n_groups=8, topk_groups=4, group_topn=2) if grouped else dict()
+    # skewed scores so that the capacity binds
+    s = (g.random((T, N)) * np.linspace(1.0, 0.2, N)[None, :]).astype(np.float32)
+    b = g.uniform(-0.01, 0.01, N).astype(np.float32)
+    idx, w, info = orc.route_capacity(s, b, K, scale=2.5, **kw)
+    C = info["capacity"]
+    prim, _ = orc.select(s, b, K, **kw)
+    wide, _ = orc.select(s, b, 2 * K, **kw)
+    assert np.array_equal(wide[:, :K], prim)
+    _, _, _, rank, _ = orc.positions(prim, N)
+    keep = rank < C
+    assert info["overflow"] == int((~keep).sum()) > 0
+    assert np.array_equal(idx[keep], prim[keep])
+    for t in range(T):
+        j = 0
+        for k in range(K):
+            if keep[t, k]:
+                continue
+            assert idx[t, k] in (-1, wide[t, K + j])
+            j += 1
+    assert info["rerouted"] + info["dropped"] == info["overflow"]
+    assert int((idx == -1).sum()) == info["dropped"]
+    assert orc.histogram(idx, N).max() <= C
+    for t in range(T):
+        row = idx[t]
+        kept = row[row >= 0]
+        assert len(set(kept.tolist())) == len(kept)
+        if len(kept):
+            assert float(w[t][row >= 0].sum()) == pytest.approx(2.5, rel=1e-5)
+        assert (w[t][row < 0] == 0).all()
