@@ -18,6 +18,10 @@ cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const floa
                              int T, int d, int N, int fn, float* scores, cudaStream_t st);
 cudaError_t launch_bias_update_ema(const int32_t* counts, int N, int64_t total, float u, float alpha, float* ema,
                                    float* bias, cudaStream_t st);
+size_t capacity_workspace_bytes(int64_t T, int K, int N);
+cudaError_t launch_route_capacity(const float* scores, const float* bias, int T, int N, int K, int n_groups,
+                                  int topk_groups, int group_topn, int renorm, float route_scale, long long C,
+                                  int32_t* idx, float* w, long long* info, void* ws, cudaStream_t st);
 cudaError_t launch_route_balanced(int64_t T, int K, int N, float scale, int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K, int n_groups,
                               int topk_groups, int group_topn, int renorm, float route_scale, int32_t* idx,
@@ -156,6 +160,33 @@ moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t
     if (ws_bytes < moe_workspace_bytes(T, K, N, n_slots)) return MOE_ERR_INVALID;
     return cuda_status(launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets, rank,
                                          scores, score_fn, stats, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_capacity_workspace_bytes(int64_t T, int32_t K, int32_t N) {
+    if (T < 0 || K <= 0 || N <= 0) return 0;
+    return capacity_workspace_bytes(T, K, N);
+}
+
+moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, const float* bias, int64_t capacity,
+                              int32_t* topk_idx, float* topk_w, moe_capacity_info* info, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_route_cfg(cfg);
+    if (s != MOE_OK) return s;
+    const moe_route_cfg& c = *cfg;
+    if (c.K > 16 || capacity < 0) return MOE_ERR_INVALID;
+    if (c.T > 0 && (scores == nullptr || topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID;
+    if (scores != nullptr && !aligned16(scores)) return MOE_ERR_INVALID;
+    if (ws == nullptr || ws_bytes < moe_capacity_workspace_bytes(c.T, c.K, c.N)) return MOE_ERR_INVALID;
+    // the counters are always written: to info, or else to the workspace header
+    static_assert(sizeof(moe_capacity_info) == 4 * sizeof(long long), "info layout");
+    long long* inf = info != nullptr ? reinterpret_cast<long long*>(info)
+                                     : reinterpret_cast<WsHeader*>(static_cast<char*>(ws) +
+                                                                   ws_layout(c.T, c.K, c.N, c.N).header)->cap_info;
+    const int eff_topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
+    return cuda_status(launch_route_capacity(scores, c.bias_mode == 1 ? nullptr : bias, (int)c.T, c.N, c.K,
+                                             c.n_groups, eff_topk_groups, c.group_topn, c.renorm ? 1 : 0,
+                                             c.route_scale, capacity, topk_idx, topk_w, inf, ws,
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale, int32_t* topk_idx,

@@ -34,7 +34,9 @@ constexpr unsigned FULL = 0xffffffffu;
 // ---------------------------------------------------------------------------
 struct WsHeader {
     int32_t gate_err;       // bit 0: a barrier wait of the gate GEMM ran out
-    int32_t pad[63];
+    int32_t pad0;
+    long long cap_info[4];  // capacity routing counters when the caller passes none
+    int32_t pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

@@ -9,6 +9,9 @@
 // reads K expert rows and writes one (combine).  Every warp-wide access is a
 // contiguous 512-byte span, so HBM sees full lines; the row destinations
 // come from pos = offsets[slot] + rank, computed once per token by K lanes.
+// An assignment dropped by the capacity limit (slot < 0) has pos -1 and no
+// row of its own (dispatch parks its copy in the unused last row of the
+// buffer); combine skips it.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -68,9 +71,14 @@ __global__ void __launch_bounds__(DC_THREADS) dispatch_kernel(
         int my_pos = 0;
         if (lane < K) {
             const int64_t a = t * K + lane;
-            my_pos = __ldg(offsets + __ldg(slot_idx + a)) + __ldg(rank + a);
-            if (pos_out) pos_out[a] = my_pos;
-            if (row_src) row_src[my_pos] = (int32_t)t;
+            const int sl = __ldg(slot_idx + a);
+            const int q = sl >= 0 ? __ldg(offsets + sl) + __ldg(rank + a) : -1;
+            if (pos_out) pos_out[a] = q;
+            if (row_src && q >= 0) row_src[q] = (int32_t)t;
+            // a dropped assignment's copy goes to the last row, which is past
+            // the kept rows whenever anything was dropped: the store loop
+            // stays free of per-row tests
+            my_pos = q >= 0 ? q : (int)(T * K - 1);
         }
         int p[KMAX];
 #pragma unroll
@@ -140,16 +148,32 @@ __global__ void __launch_bounds__(DC_THREADS) combine_kernel(const char* __restr
                                                              int K, const int32_t* __restrict__ pos,
                                                              const float* __restrict__ w,
                                                              char* __restrict__ out) {
-    const int lane = threadIdx.x & 31;
+    __shared__ int s_pos[DC_WARPS][32];
+    __shared__ float s_w[DC_WARPS][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row_bytes = (int64_t)d * (16 / EPV);
     const int nvec = d / EPV;
-    for (int64_t t = (int64_t)blockIdx.x * DC_WARPS + (threadIdx.x >> 5); t < T;
-         t += (int64_t)gridDim.x * DC_WARPS) {
-        int my_pos = 0;
+    for (int64_t t = (int64_t)blockIdx.x * DC_WARPS + warp; t < T; t += (int64_t)gridDim.x * DC_WARPS) {
+        int my_pos = -1;
         float my_w = 0.f;
         if (lane < K) {
             my_pos = __ldg(pos + t * K + lane);
             my_w = __ldg(w + t * K + lane);
+        }
+        // the token's kept assignments (pos >= 0; dropped ones have no row)
+        // moved to the front in k order, so the sum runs over them alone
+        const unsigned live = __ballot_sync(FULL, my_pos >= 0);
+        const int Kl = __popc(live);
+        if (live != ((K >= 32) ? FULL : ((1u << K) - 1u))) {
+            if (my_pos >= 0) {
+                const int r = __popc(live & lanemask_lt());
+                s_pos[warp][r] = my_pos;
+                s_w[warp][r] = my_w;
+            }
+            __syncwarp();
+            my_pos = lane < Kl ? s_pos[warp][lane] : 0;
+            my_w = lane < Kl ? s_w[warp][lane] : 0.f;
+            __syncwarp();
         }
         for (int v0 = 0; v0 < nvec; v0 += 64) {
             float acc[2][EPV];
@@ -157,7 +181,7 @@ __global__ void __launch_bounds__(DC_THREADS) combine_kernel(const char* __restr
             for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int i = 0; i < EPV; ++i) acc[u][i] = 0.f;
-            for (int k0 = 0; k0 < K; k0 += 4) {
+            for (int k0 = 0; k0 < Kl; k0 += 4) {
                 uint4 val[4][2];
                 float wk[4];
 #pragma unroll
@@ -168,12 +192,12 @@ __global__ void __launch_bounds__(DC_THREADS) combine_kernel(const char* __restr
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int v = v0 + u * 32 + lane;
-                        if (k < K && v < nvec) ld_vec(y + (int64_t)pk * row_bytes + (int64_t)v * 16, val[kk][u]);
+                        if (k < Kl && v < nvec) ld_vec(y + (int64_t)pk * row_bytes + (int64_t)v * 16, val[kk][u]);
                     }
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    if (k0 + kk >= K) break;
+                    if (k0 + kk >= Kl) break;
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int v = v0 + u * 32 + lane;

@@ -123,7 +123,7 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, i
         }
         run += c8[j];
     }
-    if (tid == 0) offsets[n_slots] = (int)A;
+    if (tid == 0) offsets[n_slots] = total_i;  // T*K less the dropped assignments
     if (stats == nullptr) return;
     const double total = (double)total_i;
     const double mean = n_slots > 0 ? total / (double)n_slots : 0.0;
@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
         const int64_t a = base_a + j * 32 + lane;
         int slot = slot_r[j];
         if (a < A) {
-            if (slot < 0 || slot >= N) {
+            if (slot < 0) {
+                slot = -1;  // dropped by the capacity limit: no slot, rank -1
+            } else if (slot >= N) {
                 bad = 1;
                 slot = -1;
             } else if (replica_slot != nullptr) {

@@ -18,6 +18,8 @@
 
 namespace moe {
 
+int route_epl(int N);
+
 
 // Warp-wide argmax over lanes [base, base+width) by (key desc, idx asc);
 // `width` a power of two; all lanes of the span end with the winner.
@@ -51,6 +53,35 @@ __device__ __forceinline__ void load_row(const float* __restrict__ row, int lane
     }
 }
 
+// Mask of this lane's experts that are candidates: all of them without
+// groups; with groups, those of the topk_groups best groups, a group's score
+// being the fp32 sum, largest first, of its group_topn largest keys.
+template <int EPL>
+__device__ __forceinline__ unsigned kept_experts(const float (&key)[EPL], unsigned exist, int lane, int e0,
+                                                 int n_groups, int topk_groups, int group_topn, int lpg) {
+    if (n_groups <= 1) return exist;
+    unsigned left = exist;
+    float gsum = 0.f;
+    for (int r = 0; r < group_topn; ++r) {
+        float bk = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (((left >> i) & 1u) && beats(key[i], e0 + i, bk, bi)) { bk = key[i]; bi = e0 + i; }
+        argmax_span(bk, bi, lpg);
+        if (bi >= e0 && bi < e0 + EPL) left &= ~(1u << (bi - e0));
+        gsum = (r == 0) ? bk : __fadd_rn(gsum, bk);
+    }
+    // rank of my group among all groups by (score desc, group asc)
+    const int g = lane / lpg;
+    int rank = 0;
+    for (int h = 0; h < n_groups; ++h) {
+        float gh = __shfl_sync(FULL, gsum, h * lpg);
+        if (h != g && beats(gh, h, gsum, g)) ++rank;
+    }
+    return rank < topk_groups ? exist : 0u;
+}
+
 template <int EPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(
     const float* __restrict__ scores, const float* __restrict__ bias, int T, int N, int K,
@@ -75,30 +106,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 #pragma unroll
         for (int i = 0; i < EPL; ++i) key[i] = __fadd_rn(s[i], b[i]);
 
-        unsigned avail = exist;
-        if (n_groups > 1) {
-            // group score: fp32 sum, largest first, of the group's group_topn largest keys
-            unsigned left = exist;
-            float gsum = 0.f;
-            for (int r = 0; r < group_topn; ++r) {
-                float bk = -INFINITY;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i)
-                    if (((left >> i) & 1u) && beats(key[i], e0 + i, bk, bi)) { bk = key[i]; bi = e0 + i; }
-                argmax_span(bk, bi, lpg);
-                if (bi >= e0 && bi < e0 + EPL) left &= ~(1u << (bi - e0));
-                gsum = (r == 0) ? bk : __fadd_rn(gsum, bk);
-            }
-            // rank of my group among all groups by (score desc, group asc)
-            const int g = lane / lpg;
-            int rank = 0;
-            for (int h = 0; h < n_groups; ++h) {
-                float gh = __shfl_sync(FULL, gsum, h * lpg);
-                if (h != g && beats(gh, h, gsum, g)) ++rank;
-            }
-            if (rank >= topk_groups) avail = 0;
-        }
+        unsigned avail = kept_experts<EPL>(key, exist, lane, e0, n_groups, topk_groups, group_topn, lpg);
 
         // K rounds of warp argmax over the available candidates
         float ssum = 0.f, my_s = 0.f;
@@ -126,6 +134,84 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
 }
 
+
+// Ranked candidates for capacity-limited routing ("MoE Routing Entropy vs
+// Expert Saturation", section "Production Testing": the excess goes to
+// secondary candidates).  One warp per token, 2K rounds of warp argmax by
+// (key desc, index asc) over the kept groups' experts: rounds 0..K-1 are the
+// selection (idx, in order), rounds K..2K-1 the secondaries (second, -1 once
+// the kept experts run out).  Block 0 also resets the capacity counters.
+template <int EPL>
+__global__ void __launch_bounds__(256) capacity_candidates_kernel(
+    const float* __restrict__ scores, const float* __restrict__ bias, int T, int N, int K, int n_groups,
+    int topk_groups, int group_topn, int lpg, int32_t* __restrict__ idx, int32_t* __restrict__ second,
+    long long* __restrict__ info, long long capacity) {
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int e0 = lane * EPL;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        info[0] = capacity;
+        info[1] = 0;
+        info[2] = 0;
+        info[3] = 0;
+    }
+    float b[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) b[i] = (bias != nullptr && e0 + i < N) ? __ldg(bias + e0 + i) : 0.f;
+    unsigned exist = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) if (e0 + i < N) exist |= 1u << i;
+
+    for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T; t += gridDim.x * warps_per_block) {
+        float s[EPL], key[EPL];
+        load_row<EPL>(scores + (size_t)t * N, lane, N, s);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) key[i] = __fadd_rn(s[i], b[i]);
+        unsigned avail = kept_experts<EPL>(key, exist, lane, e0, n_groups, topk_groups, group_topn, lpg);
+        int my_idx = -1;
+        for (int r = 0; r < 2 * K; ++r) {
+            float bk = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (((avail >> i) & 1u) && beats(key[i], e0 + i, bk, bi)) { bk = key[i]; bi = e0 + i; }
+            argmax_span(bk, bi, 32);
+            if (bi == 0x7fffffff) break;  // no kept expert left (uniform across the warp)
+            if (lane == bi / EPL) avail &= ~(1u << (bi - e0));
+            if (lane == r) my_idx = bi;
+        }
+        if (lane < K) idx[(size_t)t * K + lane] = my_idx;
+        else if (lane < 2 * K) second[(size_t)t * K + (lane - K)] = my_idx;
+    }
+}
+
+cudaError_t launch_capacity_candidates(const float* scores, const float* bias, int T, int N, int K, int n_groups,
+                                       int topk_groups, int group_topn, int32_t* idx, int32_t* second,
+                                       long long* info, long long capacity, cudaStream_t st) {
+    const int epl = route_epl(N);
+    const int gsize = N / n_groups;
+    const int lpg = n_groups > 1 ? gsize / epl : 32;
+    long long blocks = ((long long)T + 7) / 8;
+    const long long cap = (long long)moe_host::sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+#define MOE_CAND_CASE(E)                                                                               \
+    case E:                                                                                            \
+        capacity_candidates_kernel<E><<<(unsigned)blocks, 256, 0, st>>>(                               \
+            scores, bias, T, N, K, n_groups, topk_groups, group_topn, lpg, idx, second, info, capacity); \
+        break;
+    switch (epl) {
+        MOE_CAND_CASE(1)
+        MOE_CAND_CASE(2)
+        MOE_CAND_CASE(4)
+        MOE_CAND_CASE(8)
+        MOE_CAND_CASE(16)
+        default: return cudaErrorInvalidValue;
+    }
+#undef MOE_CAND_CASE
+    moe_host::note_launch();
+    return cudaGetLastError();
+}
 
 // ---------------------------------------------------------------------------
 // Filtered selection: S = N/32 threads per token, thread j owning experts

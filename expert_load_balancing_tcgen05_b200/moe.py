@@ -29,7 +29,7 @@ MOE_F32, MOE_BF16 = 0, 1
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
            "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout", "moe_route_balanced",
-           "moe_bias_update_ema")
+           "moe_bias_update_ema", "moe_route_capacity", "moe_capacity_workspace_bytes")
 
 
 class RouteCfg(ctypes.Structure):
@@ -135,6 +135,39 @@ _lib.moe_route_balanced.argtypes = [_I64, _I32, _I32, _F32, _P, _P, _P]
 _lib.moe_route_balanced.restype = _I32
 _lib.moe_bias_update_ema.argtypes = [_P, _I32, _I64, _F32, _F32, _P, _P, _P]
 _lib.moe_bias_update_ema.restype = _I32
+
+
+_lib.moe_capacity_workspace_bytes.argtypes = [_I64, _I32, _I32]
+_lib.moe_capacity_workspace_bytes.restype = ctypes.c_size_t
+_lib.moe_route_capacity.argtypes = [ctypes.POINTER(RouteCfg), _P, _P, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.moe_route_capacity.restype = _I32
+
+
+def capacity_limit(T, K, N):
+    """ceil(1.25 * T*K/N): the per-expert token capacity of the "Production
+    Testing" section of the entropy page, in integers."""
+    return (5 * T * K + 4 * N - 1) // (4 * N)
+
+
+def capacity_workspace(T, K, N, device="cuda"):
+    """Zero-filled workspace for moe_route_capacity (reuse it across calls)."""
+    n = _lib.moe_capacity_workspace_bytes(T, K, N)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def empty_capacity_info(device="cuda"):
+    return torch.zeros(4, dtype=torch.int64, device=device)
+
+
+def read_capacity_info(info) -> dict:
+    v = info.cpu().tolist()
+    return dict(capacity=v[0], overflow=v[1], rerouted=v[2], dropped=v[3])
+
+
+def moe_route_capacity(cfg, scores, bias, capacity, topk_idx, topk_w, info, ws, stream=None):
+    _check(_lib.moe_route_capacity(ctypes.byref(cfg), _ptr(scores), _ptr(bias), int(capacity), _ptr(topk_idx),
+                                   _ptr(topk_w), _ptr(info), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)), "moe_route_capacity")
 
 
 def moe_route_balanced(T, K, N, route_scale, topk_idx, topk_w, stream=None):

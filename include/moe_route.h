@@ -149,6 +149,45 @@ moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale
                               float* topk_w, moe_stream_t stream);
 
 /*
+ * moe_route_capacity -- capacity-limited selection ([ENT] "Production
+ * Testing": a hard token capacity per expert, 1.25 * T*K/N, with the excess
+ * routed to secondary candidate experts by the bias-adjusted ranking).
+ *   Candidates of token t: the experts of its kept groups ranked by (key
+ *   desc, index asc), key = fp32(s + bias) as in moe_route (the key is s
+ *   itself when cfg->bias_mode = 1 or bias is NULL); the first K are
+ *   moe_route's choice, in its order.
+ *   1. In flat order a = t*K + k a primary is kept while its expert has kept
+ *      fewer than `capacity`; the others overflow.
+ *   2. Token t's j-th overflowed slot (in k order) moves to its candidate
+ *      K + j, if it has one; in flat order again such a reroute is kept while
+ *      its expert holds fewer than `capacity` in all.  Everything else is
+ *      dropped: topk_idx = -1, topk_w = 0 (one reroute round).
+ *   3. Weights as in moe_route, over the token's kept slots in k order.
+ * scores [T,N] fp32 (moe_route's scores), bias [N] fp32 or NULL; cfg gives T,
+ * N, K (<= 16), the groups, renorm and route_scale (d, score_fn, in_dtype are
+ * not used).  capacity >= 0 (ceil(1.25*T*K/N) for the page's rule).
+ * topk_idx, topk_w [T,K] out; info (device, may be NULL) receives the
+ * capacity and the overflow / reroute / drop counts.  ws: a zero-filled
+ * workspace of moe_capacity_workspace_bytes() bytes, kept between calls.
+ * Six launches (candidates, two load-statistics passes, reroute, finalize);
+ * every decision comes from stable ranks, so the result equals the
+ * sequential walk and is deterministic.
+ */
+typedef struct moe_capacity_info {
+    int64_t capacity;
+    int64_t n_overflow;  /* primaries over the capacity */
+    int64_t n_rerouted;  /* of those, kept on a secondary expert */
+    int64_t n_dropped;   /* n_overflow - n_rerouted */
+} moe_capacity_info;
+
+size_t moe_capacity_workspace_bytes(int64_t T, int32_t K, int32_t N);
+
+moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, const float* bias,
+                              int64_t capacity, int32_t* topk_idx, float* topk_w,
+                              moe_capacity_info* info, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/*
  * moe_load_stats -- load histogram, expert offsets, stable in-expert ranks
  * and load statistics.
  *
@@ -156,8 +195,11 @@ moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale
  * slot id in [N, n_slots) or -1 per expert), the replica slot for odd t and
  * the original for even t ([HD] redundant experts for prefill; [GL] section
  * 2).  slot_idx [T,K] receives slot(t,k) (may be NULL).
+ * A negative topk_idx entry is an assignment dropped by the capacity limit
+ * (moe_route_capacity): it has slot -1 and rank -1 and counts nowhere.
  * counts [n_slots]: c_e = #{(t,k) : slot = e}  ([ENT] bincount).
- * offsets [n_slots + 1]: exclusive prefix of counts, offsets[n_slots] = T*K.
+ * offsets [n_slots + 1]: exclusive prefix of counts; offsets[n_slots] = the
+ *   kept assignments (T*K less the dropped ones).
  * rank [T,K]: number of earlier flat assignments (t',k') < (t,k) with the
  *   same slot -- the row's place inside its expert's segment.
  * stats (device, may be NULL): see moe_stats.  scores [T,N] fp32 (may be
@@ -226,6 +268,9 @@ moe_status moe_bias_update_ema(const int32_t* counts, int32_t N, int64_t total_a
  *   q = e4m3_rn_satfinite(fp32(v * inv)), scale = fp32(amax / 448).
  * slot_idx, offsets, rank as produced by moe_load_stats.  d % 8 == 0
  * (bf16) or d % 4 == 0 (fp32).
+ * Dropped assignments (slot_idx < 0, from moe_route_capacity) get pos = -1
+ * and no row; the buffers still hold T*K rows, and the rows from
+ * offsets[n_slots] on are scratch (the dropped copies land in the last one).
  */
 moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, int32_t K,
                         const int32_t* slot_idx, const int32_t* offsets, const int32_t* rank,
@@ -236,8 +281,9 @@ moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, in
  * moe_combine -- weighted gather-sum of expert outputs back to token order
  * ([HD] "Token routing": outputs summed weighted by affinity; "DeepEP":
  * combine, BF16).
- *   out[t, :] = sum_{k=0..K-1} w[t,k] * y[pos[t,k], :]
- * accumulated in fp32 in k order, rounded once to the output dtype.
+ *   out[t, :] = sum_{k=0..K-1, pos[t,k] >= 0} w[t,k] * y[pos[t,k], :]
+ * accumulated in fp32 in k order, rounded once to the output dtype (pos < 0:
+ * an assignment dropped by the capacity limit, skipped).
  * y [T*K, d] and out [T, d] in `dtype`; pos [T,K] int32, w [T,K] fp32.
  */
 moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32_t K,

@@ -106,6 +106,20 @@ def test_balanced_and_ema_reject_bad_arguments(moe):
     assert L.moe_bias_update_ema(FAKE, 256, 100, 0.001, 0.9, None, FAKE, None) == 1
 
 
+def test_route_capacity_rejects_bad_arguments(moe):
+    L = moe._lib
+    ws = L.moe_capacity_workspace_bytes(64, 8, 256)
+    assert ws > L.moe_workspace_bytes(64, 8, 256, 256)
+    cfg = _cfg(moe)
+    assert L.moe_route_capacity(ctypes.byref(cfg), FAKE, None, -1, FAKE, FAKE, None, FAKE, ws, None) == 1
+    assert L.moe_route_capacity(ctypes.byref(_cfg(moe, K=17, n_groups=1)), FAKE, None, 5, FAKE, FAKE, None, FAKE,
+                                ws, None) == 1
+    assert L.moe_route_capacity(ctypes.byref(cfg), None, None, 5, FAKE, FAKE, None, FAKE, ws, None) == 1
+    assert L.moe_route_capacity(ctypes.byref(cfg), FAKE, None, 5, FAKE, FAKE, None, FAKE, ws - 1, None) == 1
+    assert L.moe_route_capacity(ctypes.byref(cfg), MISALIGNED, None, 5, FAKE, FAKE, None, FAKE, ws, None) == 1
+    assert L.moe_route_capacity(None, FAKE, None, 5, FAKE, FAKE, None, FAKE, ws, None) == 1
+
+
 def test_load_stats_rejects_bad_arguments(moe):
     L = moe._lib
     ws = 1 << 24
