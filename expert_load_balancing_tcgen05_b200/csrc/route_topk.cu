@@ -239,7 +239,7 @@ cudaError_t launch_capacity_candidates(const float* scores, const float* bias, i
 constexpr int SEL_THREADS = 256;
 
 template <int S>
-__global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
+__global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
     const float* __restrict__ scores, const float* __restrict__ bias, int T, int K, int grouped,
     int topk_groups, int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w) {
@@ -263,23 +263,29 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
     for (int64_t t0 = (int64_t)blockIdx.x * TPB; t0 < T; t0 += (int64_t)gridDim.x * TPB) {
         const int64_t t = t0 + lt;
         const bool live = t < T;
-        float s[32];
+        // the keys stay in registers; the few survivors' unbiased scores are
+        // re-read (L1 hits) when they are compacted
+        const float* my_row = scores + t * N + 32 * j;
+        float kv[32];
         if (live) {
-            const float4* src = reinterpret_cast<const float4*>(scores + t * N + 32 * j);
+            const float4* src = reinterpret_cast<const float4*>(my_row);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 f = __ldg(src + q);
-                s[4 * q] = f.x; s[4 * q + 1] = f.y; s[4 * q + 2] = f.z; s[4 * q + 3] = f.w;
+                kv[4 * q] = __fadd_rn(f.x, bj[4 * q]);
+                kv[4 * q + 1] = __fadd_rn(f.y, bj[4 * q + 1]);
+                kv[4 * q + 2] = __fadd_rn(f.z, bj[4 * q + 2]);
+                kv[4 * q + 3] = __fadd_rn(f.w, bj[4 * q + 3]);
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] = 0.f;
+            for (int i = 0; i < 32; ++i) kv[i] = bj[i];
         }
         // 1. two largest keys of my 32 experts
         float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float key = __fadd_rn(s[i], bj[i]);
+            const float key = kv[i];
             t2 = key > t1 ? t1 : (key > t2 ? key : t2);
             t1 = key > t1 ? key : t1;
         }
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
         unsigned m = 0;
         if (cand) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) m |= (__fadd_rn(s[i], bj[i]) >= th ? 1u : 0u) << i;
+            for (int i = 0; i < 32; ++i) m |= (kv[i] >= th ? 1u : 0u) << i;
         }
         int total = __popc(m);
 #pragma unroll
@@ -316,7 +322,7 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
             if (cand) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float key = __fadd_rn(s[i], bj[i]);
+                    const float key = kv[i];
                     const bool g1 = key > q4[0], g2 = key > q4[1], g3 = key > q4[2], g4 = key > q4[3];
                     q4[3] = g3 ? q4[2] : (g4 ? key : q4[3]);
                     q4[2] = g2 ? q4[1] : (g3 ? key : q4[2]);
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
                 m = 0;
                 if (cand) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) m |= (__fadd_rn(s[i], bj[i]) >= th ? 1u : 0u) << i;
+                    for (int i = 0; i < 32; ++i) m |= (kv[i] >= th ? 1u : 0u) << i;
                 }
             }
             total = __popc(m);
@@ -366,8 +372,8 @@ __global__ void __launch_bounds__(SEL_THREADS) route_select_kernel(
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 if ((m >> i) & 1u) {
-                    c_key[lt][off] = __fadd_rn(s[i], bj[i]);
-                    c_s[lt][off] = s[i];
+                    c_key[lt][off] = kv[i];
+                    c_s[lt][off] = __ldg(my_row + i);
                     c_idx[lt][off] = 32 * j + i;
                     ++off;
                 }
