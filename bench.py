@@ -13,6 +13,12 @@ keep 4, bias, weights x2.5):
 Combine is timed in its own loop (identity experts: it gathers the
 dispatched rows back) and reported under "stages".
 
+Schedule: by default the steps are software-pipelined -- the routing of batch
+i+1 runs on a high-priority stream beside the dispatch of batch i (see
+expert_load_balancing_tcgen05_b200/step.py); the results are those of the
+serial order.  --serial times the calls one after another instead.  The
+per-stage times under "stages" always come from the serial schedule.
+
 Metric: routed tokens/s = tokens of all ranks / max-over-ranks device time.
 Inputs are synthetic (seeded, drawn on the device) and larger than L2, so no
 flush is needed between steps.  Rank 0 prints one JSON line.
@@ -123,95 +129,13 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------
-class Pipeline:
-    """Device buffers and the sequence of library calls of one step."""
-
-    def __init__(self, wl, rank: int, device, world: int = 1):
-        import torch
-        from expert_load_balancing_tcgen05_b200 import moe
-        from expert_load_balancing_tcgen05_b200 import workloads as W
-        self.moe, self.wl, self.dev = moe, wl, device
-        T, d, N, K = wl.T, wl.d, wl.N, wl.K
-        inp = W.make_inputs(wl, device=device, seed=wl.seed + 100 * rank)
-        self.x, self.W, self.bias0 = inp["x"], inp["W"], inp["bias"]
-        self.bias = self.bias0.clone()
-        self.off = inp["off"]
-        f32, i32 = torch.float32, torch.int32
-        self.scores = torch.empty(T, N, dtype=f32, device=device)
-        self.idx = torch.empty(T, K, dtype=i32, device=device)
-        self.w = torch.empty(T, K, dtype=f32, device=device)
-        self.slot = torch.empty(T, K, dtype=i32, device=device)
-        self.counts = torch.empty(N, dtype=i32, device=device)
-        self.offsets = torch.empty(N + 1, dtype=i32, device=device)
-        self.rank = torch.empty(T, K, dtype=i32, device=device)
-        self.pos = torch.empty(T, K, dtype=i32, device=device)
-        self.stats = moe.empty_stats(device)
-        self.ws = moe.workspace(T, K, N, N, device=device)
-        self.rows = torch.empty(T * K, d, dtype=torch.bfloat16, device=device)
-        self.out = torch.empty(T, d, dtype=torch.bfloat16, device=device)
-        self.cfg = moe.route_cfg(T, d, N, K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm,
-                                 wl.scale, moe.MOE_BF16)
-        # data-parallel: the bias is shared, so its step uses the global
-        # counts (one all-reduce of N int32), on a side stream that overlaps
-        # the dispatch; the next step's routing waits for it
-        self.world = world
-        if world > 1:
-            self.side = torch.cuda.Stream(device=device)
-            self.stats_done = torch.cuda.Event()
-            self.bias_ready = torch.cuda.Event()
-
-    def route(self, x=None):
-        self.moe.moe_route(self.cfg, self.x if x is None else x, self.W, self.off, self.bias, self.scores, self.idx,
-                           self.w, self.ws)
-
-    def load_stats(self):
-        wl = self.wl
-        self.moe.moe_load_stats(self.idx, wl.T, wl.K, wl.N, None, wl.N, self.slot, self.counts, self.offsets,
-                                self.rank, None, wl.fn, self.stats, self.ws)
-
-    def bias_update(self):
-        if self.world == 1:
-            self.moe.moe_bias_update(self.counts, self.wl.N, self.wl.T * self.wl.K, 0.001, 0, self.bias)
-            return
-        import torch
-        import torch.distributed as dist
-        self.stats_done.record()
-        with torch.cuda.stream(self.side):
-            self.side.wait_event(self.stats_done)
-            dist.all_reduce(self.counts, op=dist.ReduceOp.SUM)
-            self.moe.moe_bias_update(self.counts, self.wl.N, self.wl.T * self.wl.K * self.world, 0.001, 0,
-                                     self.bias, stream=self.side)
-            self.bias_ready.record(self.side)
-
-    def join_side(self):
-        """Make the current stream wait for the bias step (N > 1)."""
-        if self.world > 1:
-            import torch
-            torch.cuda.current_stream().wait_event(self.bias_ready)
-
-    def dispatch(self, x=None):
-        wl = self.wl
-        self.moe.moe_dispatch(self.x if x is None else x, wl.T, wl.d, wl.K, self.slot, self.offsets, self.rank,
-                              self.rows, None, None, self.pos, None)
-
-    def combine(self):
-        wl = self.wl
-        self.moe.moe_combine(self.rows, wl.T, wl.d, wl.K, self.pos, self.w, self.out)
-
-    def step(self, ev=None):
-        if ev is not None:
-            ev[0].record()
-        self.route()
-        if ev is not None:
-            ev[1].record()
-        self.load_stats()
-        self.bias_update()
-        if ev is not None:
-            ev[2].record()
-        self.dispatch()
-        if ev is not None:
-            ev[3].record()
-        self.join_side()
+def make_step(wl, rank, dev, world, pipelined):
+    """The routing step on this rank's batch (inputs drawn on the device)."""
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    from expert_load_balancing_tcgen05_b200.step import RoutingStep
+    inp = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank)
+    return RoutingStep(wl, inp["x"], inp["W"], inp["bias"].clone(), inp["off"], dev, world=world,
+                       pipelined=pipelined)
 
 
 def stage_bytes(wl):
@@ -227,10 +151,20 @@ def stage_bytes(wl):
     }
 
 
-def pipeline_roofline_us(wl, hbm_gbs, tflops):
+def pipeline_roofline_us(wl, hbm_gbs, tflops, overlapped=False):
+    """Serial schedule: the stages one after another, each at the slower of
+    its HBM and tensor bounds.  Overlapped schedule (routing of the next
+    batch beside the dispatch): all stages share HBM, so the bound is the
+    step's total bytes over HBM bandwidth, or the gate's tensor time if that
+    is longer."""
     b = stage_bytes(wl)
+    stages = ("gate", "topk", "hist", "dispatch")
+    if overlapped:
+        tb = sum(b[k]["bytes"] for k in stages) / (hbm_gbs * 1e9)
+        tf = b["gate"]["flops"] / (tflops * 1e12)
+        return max(tb, tf) * 1e6
     t = 0.0
-    for k in ("gate", "topk", "hist", "dispatch"):
+    for k in stages:
         tb = b[k]["bytes"] / (hbm_gbs * 1e9)
         tf = b[k].get("flops", 0) / (tflops * 1e12)
         t += max(tb, tf)
@@ -262,7 +196,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[WORKLOAD_NAME]
-    P = Pipeline(wl, rank, dev, world)
+    pipelined = not args.serial
+    P = make_step(wl, rank, dev, world, pipelined)
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
 
     def barrier():
@@ -295,14 +230,15 @@ def run_ours(args, rank, world, local_rank):
     # soak ~0.3 s so the sampler sees the loaded clock before and during timing
     soak(0.3)
 
-    E = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    E = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     moe.moe_launch_count(reset=True)
     barrier()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
+    P.fence()
     for i in range(args.steps):
-        P.step(E[i])
+        P.step(dispatch_events=E[i])
     stop.record()
     torch.cuda.synchronize()
     barrier()
@@ -310,20 +246,37 @@ def run_ours(args, rank, world, local_rank):
     # keep the sampler running over a few more steps so short timed regions still get samples
     soak(0.2)
     clocks = sampler.summarise(sampler.stop())
-
     ms = start.elapsed_time(stop)
-    t_route = statistics.mean(E[i][0].elapsed_time(E[i][1]) for i in range(args.steps))
-    t_stats = statistics.mean(E[i][1].elapsed_time(E[i][2]) for i in range(args.steps))
-    t_disp = statistics.mean(E[i][2].elapsed_time(E[i][3]) for i in range(args.steps))
+    t_disp = statistics.mean(a.elapsed_time(b) for a, b in E)
+    del P
+    torch.cuda.empty_cache()
+
+    # the serial schedule: per-stage times (route, load statistics + bias
+    # step, dispatch), the combine loop and the end-to-end leg
+    S = make_step(wl, rank, dev, world, pipelined=False)
+    for _ in range(3):
+        S.step()
+    n_stage = max(3, min(args.steps, 50))
+    SE = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage)]
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(n_stage):
+        S.step(stage_events=SE[i])
+    torch.cuda.synchronize()
+    t_route = statistics.mean(e[0].elapsed_time(e[1]) for e in SE)
+    t_stats = statistics.mean(e[1].elapsed_time(e[2]) for e in SE)
+    t_disp_serial = statistics.mean(e[2].elapsed_time(e[3]) for e in SE)
+    t_serial_step = statistics.mean(e[0].elapsed_time(e[3]) for e in SE)
 
     # combine: own loop (identity experts: gathers the dispatched rows back)
+    out_rows = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
     for _ in range(3):
-        P.combine()
+        moe.moe_combine(S.rows, wl.T, wl.d, wl.K, S.pos, S.w, out_rows)
     cs, ce = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     cs.record()
     for _ in range(args.steps):
-        P.combine()
+        moe.moe_combine(S.rows, wl.T, wl.d, wl.K, S.pos, S.w, out_rows)
     ce.record()
     torch.cuda.synchronize()
     t_comb = cs.elapsed_time(ce) / args.steps
@@ -336,20 +289,21 @@ def run_ours(args, rank, world, local_rank):
     tokens = wl.T * args.steps * world
     value = tokens / (ms_max / 1e3)
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # tokens, the routing path, D2H of the routing result (idx, weights,
-    # offsets, counts, stats); the dispatched rows stay on the device for the
-    # expert GEMMs.
-    x_host = P.x.cpu().pin_memory()
-    x_dev = torch.empty_like(P.x)
-    res = [P.idx, P.w, P.offsets, P.counts, P.stats]
+    # end to end through the public API with host buffers, serial schedule:
+    # H2D of the step's tokens, the routing path, D2H of the routing result
+    # (idx, weights, offsets, counts, stats); the dispatched rows stay on the
+    # device for the expert GEMMs.
+    x_host = S.x.cpu().pin_memory()
+    x_dev = torch.empty_like(S.x)
+    last = S.last()
+    res = [S.idx, S.w, last["offsets"], last["counts"], last["stats"]]
     res_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res]
     h2d = x_host.numel() * x_host.element_size()
     d2h = sum(r.numel() * r.element_size() for r in res)
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
         x_dev.copy_(x_host, non_blocking=True)
-        P.route(x_dev); P.load_stats(); P.bias_update(); P.dispatch(x_dev); P.join_side()
+        S.step(x_dev)
         for r, h in zip(res, res_host):
             h.copy_(r, non_blocking=True)
     torch.cuda.synchronize()
@@ -358,7 +312,7 @@ def run_ours(args, rank, world, local_rank):
     es.record()
     for _ in range(e2e_steps):
         x_dev.copy_(x_host, non_blocking=True)
-        P.route(x_dev); P.load_stats(); P.bias_update(); P.dispatch(x_dev); P.join_side()
+        S.step(x_dev)
         for r, h in zip(res, res_host):
             h.copy_(r, non_blocking=True)
     ee.record()
@@ -372,35 +326,46 @@ def run_ours(args, rank, world, local_rank):
     disp_bytes = b["dispatch"]["bytes"]
     achieved = disp_bytes / (t_disp / 1e3) / 1e9
     traffic = _traffic_for("dispatch_combine.cu", "dispatch_metric_dram.json")
-    roof_us = pipeline_roofline_us(wl, hbm, tf_burst)
+    roof_us = pipeline_roofline_us(wl, hbm, tf_burst, overlapped=pipelined)
+    ms_step = ms_max / args.steps
 
     out = None
     if rank == 0:
+        from expert_load_balancing_tcgen05_b200.step import PIPELINED_GATE_CTAS
+        schedule = ("pipelined: the routing of batch i+1 (gate on "
+                    f"{PIPELINED_GATE_CTAS} SMs, selection, load statistics, bias step) on a high-priority stream beside "
+                    "the dispatch of batch i") if pipelined else "serial: one call after another on one stream"
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(wl),
+            "config": {**workload_config(wl), "schedule": schedule,
                        "parallelism": (f"dp{world} (token shards; one all-reduce of the {wl.N} expert counts per "
-                                       "step for the shared bias, overlapped with dispatch)") if world > 1
+                                       "step for the shared bias, in the routing stream)") if world > 1
                        else "dp1 (independent token batches)"},
             "roofline": {"bound": "hbm", "kernel": "dispatch_kernel", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
-                         "bytes_per_launch": disp_bytes, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
-            "pipeline_roofline": {"time_us": roof_us, "frac": roof_us / (ms_max / args.steps * 1e3),
+                         "bytes_per_launch": disp_bytes, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                         "timed": "average dispatch launch in the timed region" +
+                                  (" (sharing the GPU with the next batch's routing)" if pipelined else "")},
+            "pipeline_roofline": {"time_us": roof_us, "frac": roof_us / (ms_step * 1e3),
                                   "tokens_per_s_at_roofline": wl.T / (roof_us / 1e6),
-                                  "rule": "sum over gate/topK/hist/dispatch of max(flops/bf16 burst peak, "
-                                          "bytes/HBM peak)"},
+                                  "rule": ("max(total bytes of gate/topK/hist/dispatch / HBM peak, gate flops / "
+                                           "bf16 burst peak): the stages overlap") if pipelined else
+                                          ("sum over gate/topK/hist/dispatch of max(flops/bf16 burst peak, "
+                                           "bytes/HBM peak)")},
             "stages": {
-                "route_ms": t_route, "load_stats_and_bias_ms": t_stats, "dispatch_ms": t_disp,
+                "serial_step_ms": t_serial_step,
+                "route_ms": t_route, "load_stats_and_bias_ms": t_stats, "dispatch_ms": t_disp_serial,
+                "dispatch_ms_in_timed_region": t_disp,
                 "combine_ms": t_comb,
                 "gate_topk_gbs_equiv": (b["gate"]["bytes"] + b["topk"]["bytes"]) / (t_route / 1e3) / 1e9,
                 "gate_tflops_lower_bound": b["gate"]["flops"] / (t_route / 1e3) / 1e12,
-                "dispatch_gbs": achieved,
+                "dispatch_gbs_serial": disp_bytes / (t_disp_serial / 1e3) / 1e9,
                 "combine_gbs": b["combine"]["bytes"] / (t_comb / 1e3) / 1e9,
             },
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps, "schedule": "serial"},
             "gpu_launches": launches,
             "clocks": clocks,
         }
@@ -494,6 +459,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial", action="store_true",
+                    help="time the serial schedule (one call after another) instead of the pipelined one")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

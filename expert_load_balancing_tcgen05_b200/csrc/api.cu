@@ -13,7 +13,7 @@ bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn);
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
                            bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
-                           cudaStream_t st);
+                           int max_ctas, cudaStream_t st);
 cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, const float* logit_bias,
                              int T, int d, int N, int fn, float* scores, cudaStream_t st);
 cudaError_t launch_bias_update_ema(const int32_t* counts, int N, int64_t total, float u, float alpha, float* ema,
@@ -79,6 +79,7 @@ static moe_status check_route_cfg(const moe_route_cfg* c) {
     if (c->T < 0 || c->N <= 0 || c->K <= 0 || c->K > c->N || c->K > 32) return MOE_ERR_INVALID;
     if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_INVALID;
     if (c->bias_mode != 0 && c->bias_mode != 1) return MOE_ERR_INVALID;
+    if (c->gate_max_ctas < 0) return MOE_ERR_INVALID;
     if (c->n_groups <= 0 || c->N % c->n_groups != 0 || c->n_groups > 32) return MOE_ERR_INVALID;
     const int gsize = c->N / c->n_groups;
     if (c->n_groups > 1) {
@@ -133,7 +134,7 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
             if (c.d % 8 != 0 || !aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID;
             e = launch_gate_tc(x, w_gate, logit_offset, bias, c.T, c.d, c.N, c.K, c.score_fn, c.n_groups,
                                eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, fused,
-                               bias_in_logits, scores, topk_idx, topk_w, &hdr->gate_err, st);
+                               bias_in_logits, scores, topk_idx, topk_w, &hdr->gate_err, c.gate_max_ctas, st);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
             if (fused) return MOE_OK;
         } else {

@@ -721,7 +721,7 @@ bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn) {
 }
 
 static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const tc::Epi& p, int32_t* err,
-                               cudaStream_t st) {
+                               int max_ctas, cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, 256, d, tc::BM)) return cudaErrorInvalidValue;
     const size_t smem = tc::PairCfg::SMEM_BYTES;
@@ -730,6 +730,7 @@ static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const
     if (e != cudaSuccess) return e;
     const int num_pairs = (T + 2 * tc::BM - 1) / (2 * tc::BM);
     int clusters = moe_host::sm_count() / 2;
+    if (max_ctas > 0 && clusters > max_ctas / 2) clusters = max_ctas / 2;
     if (clusters > num_pairs) clusters = num_pairs;
     if (clusters < 1) clusters = 1;
     kern<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);
@@ -739,7 +740,7 @@ static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const
 
 template <int BN>
 static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const tc::Epi& p, int32_t* err,
-                             cudaStream_t st) {
+                             int max_ctas, cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, BN, d, BN)) return cudaErrorInvalidValue;
     const size_t smem = tc::Cfg<BN>::SMEM_BYTES;
@@ -748,6 +749,7 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
     if (e != cudaSuccess) return e;
     const int num_tiles = (T + tc::BM - 1) / tc::BM;
     int grid = moe_host::sm_count();
+    if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
     if (grid > num_tiles) grid = num_tiles;
     if (grid < 1) grid = 1;
     kern<<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles);
@@ -758,19 +760,20 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
                            bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
-                           cudaStream_t st) {
+                           int max_ctas, cudaStream_t st) {
     tc::Epi p;
     p.bias_in_logits = bias_in_logits ? 1 : 0;
     p.off = off; p.bias = bias; p.scores = scores; p.idx = idx; p.w = w;
     p.T = T; p.fn = fn; p.K = K; p.n_groups = n_groups; p.topk_groups = topk_groups; p.group_topn = group_topn;
     p.renorm = renorm; p.fused = fused ? 1 : 0; p.scale = scale;
     switch (N) {
-        case 64: return launch_bn<64>(x, W, T, d, p, err, st);
-        case 128: return launch_bn<128>(x, W, T, d, p, err, st);
+        case 64: return launch_bn<64>(x, W, T, d, p, err, max_ctas, st);
+        case 128: return launch_bn<128>(x, W, T, d, p, err, max_ctas, st);
         case 256: {
             const char* e = getenv("MOE_GATE_PAIR");
             const bool pair = e == nullptr || e[0] != '0';
-            return pair ? launch_pair(x, W, T, d, p, err, st) : launch_bn<256>(x, W, T, d, p, err, st);
+            return pair ? launch_pair(x, W, T, d, p, err, max_ctas, st)
+                        : launch_bn<256>(x, W, T, d, p, err, max_ctas, st);
         }
         default: return cudaErrorInvalidValue;
     }

@@ -36,7 +36,7 @@ class RouteCfg(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("score_fn", ctypes.c_int32), ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
                 ("group_topn", ctypes.c_int32), ("renorm", ctypes.c_int32), ("route_scale", ctypes.c_float),
-                ("in_dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32)]
+                ("in_dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32), ("gate_max_ctas", ctypes.c_int32)]
 
 
 class Stats(ctypes.Structure):
@@ -225,9 +225,9 @@ def moe_version() -> str:
 # small conveniences (allocation of caller-owned buffers, decoding the stats struct)
 # --------------------------------------------------------------------------------------
 def route_cfg(T, d, N, K, score_fn, n_groups=1, topk_groups=1, group_topn=2, renorm=True, route_scale=1.0,
-              in_dtype=MOE_BF16, bias_in_logits=False) -> RouteCfg:
+              in_dtype=MOE_BF16, bias_in_logits=False, gate_max_ctas=0) -> RouteCfg:
     return RouteCfg(T, d, N, K, score_fn, n_groups, topk_groups, group_topn, 1 if renorm else 0,
-                    float(route_scale), in_dtype, 1 if bias_in_logits else 0)
+                    float(route_scale), in_dtype, 1 if bias_in_logits else 0, int(gate_max_ctas))
 
 
 def empty_stats(device="cuda") -> torch.Tensor:

@@ -1,0 +1,135 @@
+"""The routing step over batches of T tokens, every buffer allocated once:
+gate GEMM and scores, selection, load statistics, bias step, dispatch.
+
+Two schedules of the same library calls:
+
+* serial -- the calls in order on the caller's stream;
+* pipelined -- the routing of batch i+1 (gate, selection, load statistics,
+  bias step and, with several ranks, the all-reduce of the expert counts)
+  runs on a high-priority stream beside the dispatch of batch i on the
+  caller's stream.  Batch i+1 depends on batch i only through the bias,
+  which its routing stream updates in order, so every result equals the
+  serial schedule's.  The load-statistics outputs that dispatch reads
+  (slots, counts, offsets, ranks, stats) are double-buffered; a buffer set is
+  reused only after the dispatch that read it has finished.  The gate GEMM
+  gets a budget of SMs (``gate_max_ctas``) so that the dispatch, which is
+  bound by HBM bandwidth, keeps the rest of the GPU.
+
+Host-side orchestration only: streams, events and buffers.  Every step of the
+path runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import moe
+
+# SMs the gate GEMM may use while it runs beside a dispatch (pipelined schedule)
+PIPELINED_GATE_CTAS = 64
+
+
+class RoutingStep:
+    def __init__(self, wl, x, w_gate, bias, logit_offset, device, world: int = 1, pipelined: bool = True,
+                 gate_max_ctas: int | None = None, bias_rate: float = 0.001):
+        T, d, N, K = wl.T, wl.d, wl.N, wl.K
+        self.wl, self.dev, self.world, self.pipelined, self.u = wl, device, world, pipelined, bias_rate
+        self.x, self.W, self.bias, self.off = x, w_gate, bias, logit_offset
+        f32, i32 = torch.float32, torch.int32
+        self.scores = torch.empty(T, N, dtype=f32, device=device)
+        self.idx = torch.empty(T, K, dtype=i32, device=device)
+        self.w = torch.empty(T, K, dtype=f32, device=device)
+        self.sets = [dict(slot=torch.empty(T, K, dtype=i32, device=device),
+                          counts=torch.empty(N, dtype=i32, device=device),
+                          offsets=torch.empty(N + 1, dtype=i32, device=device),
+                          rank=torch.empty(T, K, dtype=i32, device=device),
+                          stats=moe.empty_stats(device))
+                     for _ in range(2 if pipelined else 1)]
+        self.ws = moe.workspace(T, K, N, N, device=device)
+        self.rows = torch.empty(T * K, d, dtype=x.dtype, device=device)
+        self.pos = torch.empty(T, K, dtype=i32, device=device)
+        if gate_max_ctas is None:
+            gate_max_ctas = PIPELINED_GATE_CTAS if pipelined else 0
+        self.cfg = moe.route_cfg(T, d, N, K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm,
+                                 wl.scale, moe.MOE_BF16 if x.dtype == torch.bfloat16 else moe.MOE_F32,
+                                 gate_max_ctas=gate_max_ctas)
+        self.i = 0
+        if pipelined:
+            _, highest = torch.cuda.Stream.priority_range()
+            self.route_stream = torch.cuda.Stream(device=device, priority=highest)
+            self.ev_routed = [torch.cuda.Event() for _ in range(2)]
+            self.ev_dispatched = [torch.cuda.Event() for _ in range(2)]
+        self.fence()
+
+    # ------------------------------------------------------------------ parts
+    def _route_part(self, s, x, stream, stage_events=None):
+        wl = self.wl
+        if stage_events is not None:
+            stage_events[0].record(stream)
+        moe.moe_route(self.cfg, x, self.W, self.off, self.bias, self.scores, self.idx, self.w, self.ws,
+                      stream=stream)
+        if stage_events is not None:
+            stage_events[1].record(stream)
+        moe.moe_load_stats(self.idx, wl.T, wl.K, wl.N, None, wl.N, s["slot"], s["counts"], s["offsets"], s["rank"],
+                           None, wl.fn, s["stats"], self.ws, stream=stream)
+        total = wl.T * wl.K
+        if self.world > 1:
+            # the bias is shared by every rank: its step uses the global counts
+            with torch.cuda.stream(stream):
+                dist.all_reduce(s["counts"], op=dist.ReduceOp.SUM)
+            total *= self.world
+        moe.moe_bias_update(s["counts"], wl.N, total, self.u, 0, self.bias, stream=stream)
+
+    def _dispatch_part(self, s, x, stream):
+        wl = self.wl
+        moe.moe_dispatch(x, wl.T, wl.d, wl.K, s["slot"], s["offsets"], s["rank"], self.rows, None, None, self.pos,
+                         None, stream=stream)
+
+    # ------------------------------------------------------------------ api
+    def fence(self):
+        """Order the routing stream after everything already on the caller's
+        stream (inputs written there, the start of a timed region)."""
+        if self.pipelined:
+            self.route_stream.wait_stream(torch.cuda.current_stream(self.dev))
+
+    def step(self, x=None, dispatch_events=None, stage_events=None):
+        """Enqueue one batch.  dispatch_events: optional (start, end) CUDA
+        events recorded around the dispatch on the caller's stream.
+        stage_events (serial schedule only): four events recorded before the
+        gate, after the selection, after the bias step and after the
+        dispatch."""
+        x = self.x if x is None else x
+        main = torch.cuda.current_stream(self.dev)
+        if not self.pipelined:
+            s = self.sets[0]
+            self._route_part(s, x, main, stage_events)
+            if stage_events is not None:
+                stage_events[2].record(main)
+            if dispatch_events is not None:
+                dispatch_events[0].record(main)
+            self._dispatch_part(s, x, main)
+            if dispatch_events is not None:
+                dispatch_events[1].record(main)
+            if stage_events is not None:
+                stage_events[3].record(main)
+            self.i += 1
+            return
+        b = self.i % 2
+        s = self.sets[b]
+        rs = self.route_stream
+        if self.i >= 2:
+            rs.wait_event(self.ev_dispatched[b])  # the dispatch that read this buffer set is done
+        self._route_part(s, x, rs)
+        self.ev_routed[b].record(rs)
+        main.wait_event(self.ev_routed[b])
+        if dispatch_events is not None:
+            dispatch_events[0].record(main)
+        self._dispatch_part(s, x, main)
+        if dispatch_events is not None:
+            dispatch_events[1].record(main)
+        self.ev_dispatched[b].record(main)
+        self.i += 1
+
+    def last(self):
+        """Buffer set (slots, counts, offsets, ranks, stats) of the last batch."""
+        return self.sets[(self.i - 1) % len(self.sets)]

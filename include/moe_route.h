@@ -69,7 +69,12 @@ typedef struct {
     int32_t bias_mode;    /* 0: bias only in the selection key (aux-loss-free routing);
                              1: bias added to the logits before the nonlinearity, so it
                                 also shapes the weights ([ENT] "Concrete Implementation":
-                                compensated_logits = raw_logits + expert_biases); needs x */
+                                the router adds its expert biases to the raw logits);
+                                needs x */
+    int32_t gate_max_ctas; /* at most this many CTAs (SMs) for the tensor-core gate GEMM,
+                              0 = all SMs; a smaller budget leaves SMs to work running
+                              beside it on another stream (e.g. the previous batch's
+                              dispatch) */
 } moe_route_cfg;
 
 /* Load statistics of one histogram, written to device memory.

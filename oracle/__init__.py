@@ -261,8 +261,8 @@ def route(x, W, off, bias, fn, K, n_groups=1, topk_groups=1, group_topn=2, renor
 
     bias_in_logits: the bias joins the logits before the nonlinearity, as in
     the DynamicEntropyMoERouter of "MoE Routing Entropy vs Expert
-    Saturation" ("Concrete Implementation": compensated_logits = raw_logits
-    + expert_biases), so it shapes the weights too and selection uses the
+    Saturation" ("Concrete Implementation": the router adds its expert biases
+    to the raw logits), so it shapes the weights too and selection uses the
     scores themselves; otherwise it only shifts the selection key."""
     h = logits(x, W, off)
     if bias_in_logits and bias is not None:

@@ -1,0 +1,40 @@
+"""The pipelined routing step (routing of batch i+1 beside the dispatch of
+batch i, double-buffered load-statistics outputs) produces exactly what the
+serial schedule produces: the same bias after the last step, the same
+routing, offsets, ranks, statistics and dispatched rows for the last batch.
+(Intermediate biases are not compared: the routing stream may already be
+updating the next batch's bias while the caller's stream runs.)"""
+import pytest
+import torch
+
+from expert_load_balancing_tcgen05_b200 import workloads as W
+from expert_load_balancing_tcgen05_b200.step import RoutingStep
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+
+
+@pytest.mark.parametrize("name,T,steps", [("metric", 4096, 7), ("collapse", 3000, 6), ("softmax_dispatch", 2500, 5)])
+def test_pipelined_equals_serial(name, T, steps):
+    wl = W.WORKLOADS[name].with_(T=T)
+    inp = W.make_inputs(wl, device="cuda", seed=5)
+    bias0 = inp["bias"] if inp["bias"] is not None else torch.zeros(wl.N, device="cuda")
+    runs = {}
+    for pipelined in (False, True):
+        S = RoutingStep(wl, inp["x"], inp["W"], bias0.clone(), inp["off"], "cuda", pipelined=pipelined)
+        for _ in range(steps):
+            S.step()
+        torch.cuda.synchronize()
+        last = S.last()
+        runs[pipelined] = dict(bias=S.bias.clone(), idx=S.idx.clone(), w=S.w.clone(), rows=S.rows.clone(), pos=S.pos.clone(),
+                               **{k: last[k].clone() for k in ("slot", "counts", "offsets", "rank", "stats")})
+    a, b = runs[False], runs[True]
+    assert torch.equal(a["bias"], b["bias"])
+    for k in ("idx", "w", "pos", "slot", "counts", "offsets", "rank", "stats"):
+        assert torch.equal(a[k], b[k]), k
+    assert torch.equal(a["rows"].view(torch.int16), b["rows"].view(torch.int16))
