@@ -66,6 +66,7 @@ def _cfg(moe, **kw):
     (dict(topk_groups=9), 1), (dict(group_topn=33), 1), (dict(score_fn=5), 1),
     (dict(n_groups=8, topk_groups=1, K=40), 1), (dict(N=96, n_groups=1, K=8), 2),
     (dict(N=256, n_groups=64, topk_groups=8), 1), (dict(N=24, n_groups=2, topk_groups=1, K=4), 2),
+    (dict(gate_max_ctas=-1), 1), (dict(bias_mode=3), 1),
 ])
 def test_route_rejects_bad_config(moe, kw, status):
     cfg = _cfg(moe, **kw)
