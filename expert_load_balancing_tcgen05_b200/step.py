@@ -92,19 +92,38 @@ class RoutingStep:
         if self.pipelined:
             self.route_stream.wait_stream(torch.cuda.current_stream(self.dev))
 
-    def step(self, x=None, dispatch_events=None, stage_events=None):
-        """Enqueue one batch.  dispatch_events: optional (start, end) CUDA
-        events recorded around the dispatch on the caller's stream.
-        stage_events (serial schedule only): four events recorded before the
-        gate, after the selection, after the bias step and after the
-        dispatch."""
+    def results(self, s):
+        """The routing result of a batch: indices, weights, offsets, counts, stats."""
+        return [self.idx, self.w, s["offsets"], s["counts"], s["stats"]]
+
+    def _copy_out(self, s, host_out, stream):
+        with torch.cuda.stream(stream):
+            for src, dst in zip(self.results(s), host_out):
+                dst.copy_(src, non_blocking=True)
+
+    def step(self, x=None, dispatch_events=None, stage_events=None, ready=None, host_out=None):
+        """Enqueue one batch.
+
+        x: the batch's tokens (default: the ones given at construction);
+        ready: an event after which x is valid (e.g. the end of its copy from
+        the host on another stream); host_out: pinned host tensors shaped like
+        results(), filled with this batch's routing result (indices and
+        weights are copied before the next batch overwrites them).
+        dispatch_events: optional (start, end) CUDA events recorded around the
+        dispatch on the caller's stream.  stage_events (serial schedule only):
+        four events recorded before the gate, after the selection, after the
+        bias step and after the dispatch."""
         x = self.x if x is None else x
         main = torch.cuda.current_stream(self.dev)
         if not self.pipelined:
             s = self.sets[0]
+            if ready is not None:
+                main.wait_event(ready)
             self._route_part(s, x, main, stage_events)
             if stage_events is not None:
                 stage_events[2].record(main)
+            if host_out is not None:
+                self._copy_out(s, host_out, main)
             if dispatch_events is not None:
                 dispatch_events[0].record(main)
             self._dispatch_part(s, x, main)
@@ -119,7 +138,11 @@ class RoutingStep:
         rs = self.route_stream
         if self.i >= 2:
             rs.wait_event(self.ev_dispatched[b])  # the dispatch that read this buffer set is done
+        if ready is not None:
+            rs.wait_event(ready)
         self._route_part(s, x, rs)
+        if host_out is not None:
+            self._copy_out(s, host_out, rs)
         self.ev_routed[b].record(rs)
         main.wait_event(self.ev_routed[b])
         if dispatch_events is not None:

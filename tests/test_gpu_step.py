@@ -38,3 +38,37 @@ def test_pipelined_equals_serial(name, T, steps):
     for k in ("idx", "w", "pos", "slot", "counts", "offsets", "rank", "stats"):
         assert torch.equal(a[k], b[k]), k
     assert torch.equal(a["rows"].view(torch.int16), b["rows"].view(torch.int16))
+
+
+def test_pipelined_with_host_copies_equals_serial():
+    """Tokens copied from pinned host memory on a copy stream (two device
+    buffers) and routing results copied back to host: the last batch's host
+    results equal the serial schedule's device results."""
+    wl = W.WORKLOADS["metric"].with_(T=2048)
+    inp = W.make_inputs(wl, device="cuda", seed=9)
+    S = RoutingStep(wl, inp["x"], inp["W"], inp["bias"].clone(), inp["off"], "cuda", pipelined=False)
+    P = RoutingStep(wl, inp["x"], inp["W"], inp["bias"].clone(), inp["off"], "cuda", pipelined=True)
+    x_host = inp["x"].cpu().pin_memory()
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
+    host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in P.results(P.sets[0])]
+    cs = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    ev_copied = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
+    steps = 5
+    cs.wait_stream(main)
+    for i in range(steps):
+        b = i % 2
+        if i >= 2:
+            cs.wait_event(ev_free[b])
+        with torch.cuda.stream(cs):
+            x_dev[b].copy_(x_host, non_blocking=True)
+        ev_copied[b].record(cs)
+        P.step(x_dev[b], ready=ev_copied[b], host_out=host)
+        ev_free[b].record(main)
+        S.step()
+    torch.cuda.synchronize()
+    for h, d in zip(host, S.results(S.last())):
+        assert torch.equal(h, d.cpu())
+    assert torch.equal(P.rows.view(torch.int16), S.rows.view(torch.int16))
+    assert torch.equal(P.bias, S.bias)
