@@ -360,7 +360,8 @@ def run_ours(args, rank, world, local_rank):
                          "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                          "bytes_per_launch": disp_bytes, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                          "timed": "average dispatch launch in the timed region" +
-                                  (" (sharing the GPU with the next batch's routing)" if pipelined else "")},
+                                  (" (sharing the GPU with the next batch's routing)" if pipelined else ""),
+                         "frac_alone": disp_bytes / (t_disp_serial / 1e3) / 1e9 / hbm},
             "pipeline_roofline": {"time_us": roof_us, "frac": roof_us / (ms_step * 1e3),
                                   "tokens_per_s_at_roofline": wl.T / (roof_us / 1e6),
                                   "rule": ("max(total bytes of gate/topK/hist/dispatch / HBM peak, gate flops / "
@@ -467,6 +468,124 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_kernel_report():
+    """Per-call device times of the library on every workload (3 warm-up
+    calls, then 10 calls captured in a CUDA graph and replayed under CUDA
+    events), each against its bound: HBM
+    bytes over the measured copy bandwidth, or the gate's flops over the
+    measured bf16 peak if longer.  Prints a markdown table (not the
+    benchmark's JSON line)."""
+    import torch
+    from expert_load_balancing_tcgen05_b200 import moe
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    hbm, tf_burst, _, _ = _peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    def t_us(fn, n=10):
+        # n calls captured in a CUDA graph and replayed: device time, without
+        # the host's launch rate
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / n * 1e3
+
+    rows = []
+
+    def add(wl, call, us, nbytes, flops=0, note=""):
+        bound = max(nbytes / (hbm * 1e9), flops / (tf_burst * 1e12)) * 1e6
+        rows.append((wl.name, f"T={wl.T} d={wl.d} N={wl.N} K={wl.K}", call, us, bound, bound / us, note))
+
+    for name in ("tiny_softmax", "v3_router", "collapse", "softmax_dispatch", "prefill_replicas", "metric"):
+        wl = W.WORKLOADS[name]
+        T, d, N, K = wl.T, wl.d, wl.N, wl.K
+        A = T * K
+        es = 2 if wl.dtype == torch.bfloat16 else 4
+        inp = W.make_inputs(wl, device=dev, seed=wl.seed, with_y=wl.combine)
+        x, Wg, off, bias = inp["x"], inp["W"], inp["off"], inp["bias"]
+        scores = torch.empty(T, N, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        w = torch.empty(T, K, device=dev)
+        n_slots = wl.n_slots
+        ws = moe.workspace(T, K, N, n_slots, device=dev)
+        dt = moe.MOE_BF16 if wl.dtype == torch.bfloat16 else moe.MOE_F32
+        cfg = moe.route_cfg(T, d, N, K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale, dt)
+        route = lambda: moe.moe_route(cfg, x, Wg, off, bias, scores, idx, w, ws)
+        add(wl, "moe_route (gate + selection)", t_us(route), T * d * es + N * d * es + T * N * 4 + A * 8,
+            2 * T * d * N)
+        sel = lambda: moe.moe_route(cfg, None, None, None, bias, scores, idx, w, ws)
+        add(wl, "  selection alone (scores given)", t_us(sel), T * N * 4 + A * 8)
+        route()
+        slot = torch.empty(T, K, dtype=torch.int32, device=dev)
+        rank = torch.empty(T, K, dtype=torch.int32, device=dev)
+        counts = torch.empty(n_slots, dtype=torch.int32, device=dev)
+        offsets = torch.empty(n_slots + 1, dtype=torch.int32, device=dev)
+        stats = moe.empty_stats(dev)
+        rep = None
+        if wl.n_replicas:
+            moe.moe_load_stats(idx, T, K, N, None, N, slot, counts[:N], offsets[:N + 1], rank, None, wl.fn, stats,
+                               ws)
+            rep = torch.empty(N, dtype=torch.int32, device=dev)
+            moe.moe_replica_plan(counts[:N], N, wl.n_replicas, rep)
+            add(wl, "moe_replica_plan", t_us(lambda: moe.moe_replica_plan(counts[:N], N, wl.n_replicas, rep)),
+                N * 8)
+        ls = lambda: moe.moe_load_stats(idx, T, K, N, rep, n_slots, slot, counts, offsets, rank, None, wl.fn, stats,
+                                        ws)
+        add(wl, "moe_load_stats", t_us(ls), A * 12 + n_slots * 8, note="latency-bound (single-pass scan)")
+        ls()
+        if wl.bias_steps or wl.has_bias:
+            b2 = bias.clone() if bias is not None else torch.zeros(N, device=dev)
+            add(wl, "moe_bias_update", t_us(lambda: moe.moe_bias_update(counts[:N], N, A, 0.001, 0, b2)), N * 8,
+                note="one block")
+        rows_b = torch.empty(A, d, dtype=wl.dtype, device=dev)
+        pos = torch.empty(T, K, dtype=torch.int32, device=dev)
+        disp = lambda: moe.moe_dispatch(x, T, d, K, slot, offsets, rank, rows_b, None, None, pos, None)
+        add(wl, "moe_dispatch", t_us(disp), T * d * es + A * d * es + A * 12)
+        if wl.fp8:
+            q = torch.empty(A, d, dtype=torch.uint8, device=dev)
+            sc = torch.empty(A, d // 128, device=dev)
+            disp8 = lambda: moe.moe_dispatch(x, T, d, K, slot, offsets, rank, rows_b, q, sc, pos, None)
+            add(wl, "moe_dispatch + FP8 copy", t_us(disp8), T * d * es + A * d * (es + 1) + A * d // 32 + A * 12)
+            del q, sc
+        disp()
+        y = inp.get("y")
+        if y is None:
+            y = rows_b
+        out = torch.empty(T, d, dtype=wl.dtype, device=dev)
+        comb = lambda: moe.moe_combine(y, T, d, K, pos, w, out)
+        add(wl, "moe_combine", t_us(comb), A * d * es + A * 8 + T * d * es)
+        if name == "metric":
+            C = moe.capacity_limit(T, K, N)
+            ci, cw = torch.empty_like(idx), torch.empty_like(w)
+            info = moe.empty_capacity_info(dev)
+            cws = moe.capacity_workspace(T, K, N, dev)
+            cap = lambda: moe.moe_route_capacity(cfg, scores, bias, C, ci, cw, info, cws)
+            add(wl, "moe_route_capacity (from scores)", t_us(cap), T * N * 4 + A * 8 * 4,
+                note="six launches, latency-bound")
+            rb = lambda: moe.moe_route_balanced(T, K, N, wl.scale, ci, cw)
+            add(wl, "moe_route_balanced", t_us(rb), A * 8)
+        del inp, x, rows_b, y, out
+        torch.cuda.empty_cache()
+
+    print(f"| workload | shape | call | time (us) | bound (us) | fraction of bound | note |")
+    print("|---|---|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r[0]} | {r[1]} | {r[2]} | {r[3]:.1f} | {r[4]:.1f} | {r[5]:.2f} | {r[6]} |")
+    print(f"\nbounds: HBM {hbm} GB/s (measured copy), bf16 {tf_burst} TFLOP/s (measured burst)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -474,6 +593,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels", action="store_true",
+                    help="print per-call device times of every workload against their bounds (markdown)")
     ap.add_argument("--serial", action="store_true",
                     help="time the serial schedule (one call after another) instead of the pipelined one")
     args = ap.parse_args()
@@ -484,6 +605,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.kernels:
+        run_kernel_report()
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

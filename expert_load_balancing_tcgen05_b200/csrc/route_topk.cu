@@ -247,8 +247,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
     constexpr int TPB = SEL_THREADS / S;       // tokens per block
     constexpr int SEL_CAP = S >= 4 ? 32 : 16;  // survivors kept per token in shared memory
     __shared__ float bias_s[N];
-    __shared__ float c_key[TPB][SEL_CAP], c_s[TPB][SEL_CAP];
-    __shared__ int c_idx[TPB][SEL_CAP];
+    // lists padded by one word: the tokens of a warp start in different banks
+    __shared__ float c_key[TPB][SEL_CAP + 1], c_s[TPB][SEL_CAP + 1];
+    __shared__ int c_idx[TPB][SEL_CAP + 1];
     __shared__ float o_s[TPB][8];
     __shared__ int o_i[TPB][8];
     for (int i = threadIdx.x; i < N; i += blockDim.x) bias_s[i] = bias != nullptr ? bias[i] : 0.f;
@@ -392,10 +393,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
                 if (rank < K) { o_i[lt][rank] = ic; o_s[lt][rank] = c_s[lt][c]; }
             }
             __syncwarp();
-            if (j == 0 && live) {
+            if (live) {
+                // every thread forms the same k-ordered sum; thread k writes slot k
                 float ssum = o_s[lt][0];
                 for (int k = 1; k < K; ++k) ssum = __fadd_rn(ssum, o_s[lt][k]);
-                for (int k = 0; k < K; ++k) {
+                for (int k = j; k < K; k += S) {
                     const float wv = renorm ? __fdiv_rn(o_s[lt][k], ssum) : o_s[lt][k];
                     topk_idx[t * K + k] = o_i[lt][k];
                     topk_w[t * K + k] = __fmul_rn(wv, route_scale);
