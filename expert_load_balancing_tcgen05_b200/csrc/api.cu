@@ -230,15 +230,15 @@ moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, in
     if (T < 0 || d <= 0 || K <= 0 || K > 32) return MOE_ERR_INVALID;
     if (T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
     if (x_dtype != MOE_BF16 && x_dtype != MOE_F32) return MOE_ERR_INVALID;
-    if (x == nullptr || slot_idx == nullptr || offsets == nullptr || rank == nullptr) return MOE_ERR_INVALID;
-    if ((rows_fp8 == nullptr) != (scales == nullptr)) return MOE_ERR_INVALID;
     const int epv = x_dtype == MOE_BF16 ? 8 : 4;
     if (d % epv != 0) return MOE_ERR_INVALID;
+    if (T == 0) return MOE_OK;  // empty batch: nothing is read or written, buffers may be NULL
+    if (x == nullptr || slot_idx == nullptr || offsets == nullptr || rank == nullptr) return MOE_ERR_INVALID;
+    if ((rows_fp8 == nullptr) != (scales == nullptr)) return MOE_ERR_INVALID;
     if (rows_fp8 != nullptr && (d % 128 != 0 || (reinterpret_cast<uintptr_t>(rows_fp8) & 7u) ||
                                 (reinterpret_cast<uintptr_t>(scales) & 3u)))
         return MOE_ERR_INVALID;
     if (!aligned16(x) || (rows != nullptr && !aligned16(rows))) return MOE_ERR_INVALID;
-    if (T == 0) return MOE_OK;
     return cuda_status(launch_dispatch(x, x_dtype, T, d, K, slot_idx, offsets, rank, rows, rows_fp8, scales, pos,
                                        row_src, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -248,10 +248,11 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
     if (T < 0 || d <= 0 || K <= 0 || K > 32) return MOE_ERR_INVALID;
     if (T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
     if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID;
-    if (y == nullptr || pos == nullptr || w == nullptr || out == nullptr) return MOE_ERR_INVALID;
     const int epv = dtype == MOE_BF16 ? 8 : 4;
-    if (d % epv != 0 || !aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID;
-    if (T == 0) return MOE_OK;
+    if (d % epv != 0) return MOE_ERR_INVALID;
+    if (T == 0) return MOE_OK;  // empty batch: buffers may be NULL
+    if (y == nullptr || pos == nullptr || w == nullptr || out == nullptr) return MOE_ERR_INVALID;
+    if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID;
     return cuda_status(launch_combine(y, dtype, T, d, K, pos, w, out, reinterpret_cast<cudaStream_t>(stream)));
 }
 

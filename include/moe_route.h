@@ -273,6 +273,7 @@ moe_status moe_bias_update_ema(const int32_t* counts, int32_t N, int64_t total_a
  *   q = e4m3_rn_satfinite(fp32(v * inv)), scale = fp32(amax / 448).
  * slot_idx, offsets, rank as produced by moe_load_stats.  d % 8 == 0
  * (bf16) or d % 4 == 0 (fp32).
+ * T = 0: nothing is read or written and every buffer may be NULL.
  * Dropped assignments (slot_idx < 0, from moe_route_capacity) get pos = -1
  * and no row; the buffers still hold T*K rows, and the rows from
  * offsets[n_slots] on are scratch (the dropped copies land in the last one).
@@ -288,7 +289,8 @@ moe_status moe_dispatch(const void* x, int32_t x_dtype, int64_t T, int32_t d, in
  * combine, BF16).
  *   out[t, :] = sum_{k=0..K-1, pos[t,k] >= 0} w[t,k] * y[pos[t,k], :]
  * accumulated in fp32 in k order, rounded once to the output dtype (pos < 0:
- * an assignment dropped by the capacity limit, skipped).
+ * an assignment dropped by the capacity limit, skipped).  T = 0: buffers may
+ * be NULL.
  * y [T*K, d] and out [T, d] in `dtype`; pos [T,K] int32, w [T,K] fp32.
  */
 moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32_t K,
