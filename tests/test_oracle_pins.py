@@ -569,3 +569,26 @@ def test_capacity_invariants(orc, grouped):
         if len(kept):
             assert float(w[t][row >= 0].sum()) == pytest.approx(2.5, rel=1e-5)
         assert (w[t][row < 0] == 0).all()
+
+
+def test_bias_update_ema_sign_follows_the_average_not_the_batch(orc):
+    # ema0 = [20, 0, 8, 4], this batch [4, 12, 8, 8] (mean 8), alpha = 0.5:
+    # ema = [12, 6, 8, 6] -> signs (+, -, 0, -) although the batch alone
+    # says (-, +, 0, 0)
+    counts = np.array([4, 12, 8, 8])
+    b, e = orc.bias_update_ema(counts, 32, np.zeros(4, np.float32), np.array([20, 0, 8, 4], np.float32), 0.001, 0.5)
+    assert e.tolist() == [12.0, 6.0, 8.0, 6.0]
+    u = np.float32(0.001)
+    assert b.tolist() == [-u, u, 0.0, u]
+
+
+def test_bias_in_logits_selects_on_the_scores_alone(orc):
+    # sigmoid, two experts, K = 1: h = (3, 2), b = (0, 0.5).  With the bias in
+    # the logits the scores are sigma(3) > sigma(2.5), so expert 0 wins; adding
+    # the bias to the key as well would pick expert 1 (sigma(2.5) + 0.5 larger)
+    x = np.array([[1.0]], np.float32)
+    W = np.array([[3.0], [2.0]], np.float32)
+    b = np.array([0.0, 0.5], np.float32)
+    _, s, idx, w = orc.route(x, W, None, b, 1, 1, bias_in_logits=True)
+    assert idx.tolist() == [[0]] and w.tolist() == [[1.0]]
+    assert s[0, 0] > s[0, 1] and s[0, 1] + b[1] > s[0, 0]
