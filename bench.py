@@ -80,7 +80,8 @@ class ClockSampler:
 
     def start(self):
         import tempfile
-        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        # inside the working tree (git-ignored), not the system temp directory
+        fd, self.path = tempfile.mkstemp(prefix=".clocks_", suffix=".csv", dir=ROOT)
         os.close(fd)
         try:
             self.f = open(self.path, "w")
@@ -462,7 +463,7 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl),
+            "config": {**workload_config(wl), "sample_tokens": n},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
