@@ -62,7 +62,8 @@ def workload_config(wl):
                         f"{wl.topk_groups}, group score top-{wl.group_topn} sum, bias U(-0.01,0.01), "
                         f"weights x{wl.scale}, bf16 x~N(0,1) W~N(0,1/d)",
             "T": wl.T, "d": wl.d, "N": wl.N, "K": wl.K, "global_batch": None,
-            "l2": "inputs larger than L2 (x 235 MB, dispatch buffer 1.88 GB per rank); no flush"}
+            "l2": "inputs larger than L2 (x 235 MB, dispatch buffer 1.88 GB per rank); consecutive steps "
+                  "alternate between two distinct token batches; no flush"}
 
 
 # --------------------------------------------------------------------------------------
@@ -131,11 +132,14 @@ class ClockSampler:
 # our arm
 # --------------------------------------------------------------------------------------
 def make_step(wl, rank, dev, world, pipelined):
-    """The routing step on this rank's batch (inputs drawn on the device)."""
+    """The routing step on this rank's batches (inputs drawn on the device).
+    Consecutive steps alternate between two distinct token batches in
+    different buffers, so that overlapped steps never share rows of x in L2."""
     from expert_load_balancing_tcgen05_b200 import workloads as W
     from expert_load_balancing_tcgen05_b200.step import RoutingStep
     inp = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank)
-    return RoutingStep(wl, inp["x"], inp["W"], inp["bias"].clone(), inp["off"], dev, world=world,
+    x2 = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank + 50)["x"]
+    return RoutingStep(wl, [inp["x"], x2], inp["W"], inp["bias"].clone(), inp["off"], dev, world=world,
                        pipelined=pipelined)
 
 

@@ -30,10 +30,16 @@ PIPELINED_GATE_CTAS = 64
 
 
 class RoutingStep:
+    """x: the token batch [T, d], or a list of batches that step() cycles
+    through when it is given none (consecutive batches then live in
+    different buffers, as in a stream of distinct batches)."""
+
     def __init__(self, wl, x, w_gate, bias, logit_offset, device, world: int = 1, pipelined: bool = True,
                  gate_max_ctas: int | None = None, bias_rate: float = 0.001):
         T, d, N, K = wl.T, wl.d, wl.N, wl.K
         self.wl, self.dev, self.world, self.pipelined, self.u = wl, device, world, pipelined, bias_rate
+        self.batches = list(x) if isinstance(x, (list, tuple)) else [x]
+        x = self.batches[0]
         self.x, self.W, self.bias, self.off = x, w_gate, bias, logit_offset
         f32, i32 = torch.float32, torch.int32
         self.scores = torch.empty(T, N, dtype=f32, device=device)
@@ -104,7 +110,8 @@ class RoutingStep:
     def step(self, x=None, dispatch_events=None, stage_events=None, ready=None, host_out=None):
         """Enqueue one batch.
 
-        x: the batch's tokens (default: the ones given at construction);
+        x: the batch's tokens (default: the next of the batches given at
+        construction);
         ready: an event after which x is valid (e.g. the end of its copy from
         the host on another stream); host_out: pinned host tensors shaped like
         results(), filled with this batch's routing result (indices and
@@ -113,7 +120,7 @@ class RoutingStep:
         dispatch on the caller's stream.  stage_events (serial schedule only):
         four events recorded before the gate, after the selection, after the
         bias step and after the dispatch."""
-        x = self.x if x is None else x
+        x = self.batches[self.i % len(self.batches)] if x is None else x
         main = torch.cuda.current_stream(self.dev)
         if not self.pipelined:
             s = self.sets[0]
