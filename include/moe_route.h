@@ -112,9 +112,14 @@ size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
  * Gate ([ENT] "The Mathematics": h = x . W_g; "Concrete Implementation":
  * nn.Linear(hidden, N, bias=False)):
  *   h[t,e] = sum_j x[t,j] * w_gate[e,j] + logit_offset[e]
- *   x [T,d], w_gate [N,d] in cfg->in_dtype (bf16: tcgen05 tensor-core GEMM
- *   with fp32 accumulation, N % 16 == 0 and N <= 256; fp32: SIMT fp32 GEMM);
- *   logit_offset [N] fp32 or NULL.
+ *   x [T,d], w_gate [N,d] in cfg->in_dtype, d % 8 == 0 for bf16.  bf16 with
+ *   N in {64, 128, 256}: tcgen05 tensor-core GEMM with fp32 accumulation
+ *   (N = 256 on a 2-SM CTA pair; environment variable MOE_GATE_PAIR=0 uses
+ *   one CTA per 128-token tile instead); other N, and fp32 inputs:
+ *   CUDA-core GEMM with fp32 accumulation.  logit_offset [N] fp32 or NULL.
+ * Shapes: N <= 32 or N in {64, 128, 256, 512}; K <= min(N, 32); groups of
+ * N / n_groups experts (n_groups <= 32) whose size is a power-of-two multiple
+ * of N / 32 when N > 32.  Other valid shapes return MOE_ERR_UNSUPPORTED.
  * Scores, fused into the GEMM epilogue, written to scores [T,N] fp32:
  *   softmax over N ([ENT] softmax equation) or sigmoid ([HD] "Token routing").
  *   If x == NULL the call skips the GEMM and reads `scores` as input instead.
