@@ -118,8 +118,8 @@ size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
  *   one CTA per 128-token tile instead); other N, and fp32 inputs:
  *   CUDA-core GEMM with fp32 accumulation.  logit_offset [N] fp32 or NULL.
  * Shapes: N <= 32 or N in {64, 128, 256, 512}; K <= min(N, 32); groups of
- * N / n_groups experts (n_groups <= 32) whose size is a power-of-two multiple
- * of N / 32 when N > 32.  Other valid shapes return MOE_ERR_UNSUPPORTED.
+ * N / n_groups experts (n_groups <= 32), a size of max(N / 32, 1) times a
+ * power of two.  Other valid shapes return MOE_ERR_UNSUPPORTED.
  * Scores, fused into the GEMM epilogue, written to scores [T,N] fp32:
  *   softmax over N ([ENT] softmax equation) or sigmoid ([HD] "Token routing").
  *   If x == NULL the call skips the GEMM and reads `scores` as input instead.
