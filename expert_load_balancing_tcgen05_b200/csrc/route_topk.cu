@@ -246,20 +246,22 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
     constexpr int N = 32 * S;
     constexpr int TPB = SEL_THREADS / S;       // tokens per block
     constexpr int SEL_CAP = S >= 4 ? 32 : 16;  // survivors kept per token in shared memory
-    __shared__ float bias_s[N];
+    // bias transposed, bias_t[i * S + j] = bias[32 * j + i]: the S threads of a
+    // token read consecutive words for the same i (no bank conflicts)
+    __shared__ float bias_t[N];
     // lists padded by one word: the tokens of a warp start in different banks
     __shared__ float c_key[TPB][SEL_CAP + 1], c_s[TPB][SEL_CAP + 1];
     __shared__ int c_idx[TPB][SEL_CAP + 1];
     __shared__ float o_s[TPB][8];
     __shared__ int o_i[TPB][8];
-    for (int i = threadIdx.x; i < N; i += blockDim.x) bias_s[i] = bias != nullptr ? bias[i] : 0.f;
+    for (int e = threadIdx.x; e < N; e += blockDim.x) bias_t[(e & 31) * S + (e >> 5)] = bias != nullptr ? bias[e] : 0.f;
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
     const int j = threadIdx.x % S;                 // which 32 experts
     const int lt = threadIdx.x / S;                // token slot in the block
     const int seg = lane - (lane % S);             // first lane of this token's segment
-    const float* bj = bias_s + 32 * j;
+    const float* bj = bias_t + j;  // bias of expert 32 j + i at bj[i * S]
 
     for (int64_t t0 = (int64_t)blockIdx.x * TPB; t0 < T; t0 += (int64_t)gridDim.x * TPB) {
         const int64_t t = t0 + lt;
@@ -273,14 +275,14 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 f = __ldg(src + q);
-                kv[4 * q] = __fadd_rn(f.x, bj[4 * q]);
-                kv[4 * q + 1] = __fadd_rn(f.y, bj[4 * q + 1]);
-                kv[4 * q + 2] = __fadd_rn(f.z, bj[4 * q + 2]);
-                kv[4 * q + 3] = __fadd_rn(f.w, bj[4 * q + 3]);
+                kv[4 * q] = __fadd_rn(f.x, bj[(4 * q) * S]);
+                kv[4 * q + 1] = __fadd_rn(f.y, bj[(4 * q + 1) * S]);
+                kv[4 * q + 2] = __fadd_rn(f.z, bj[(4 * q + 2) * S]);
+                kv[4 * q + 3] = __fadd_rn(f.w, bj[(4 * q + 3) * S]);
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) kv[i] = bj[i];
+            for (int i = 0; i < 32; ++i) kv[i] = bj[i * S];
         }
         // 1. two largest keys of my 32 experts
         float t1 = -INFINITY, t2 = -INFINITY;
@@ -411,7 +413,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
             for (int e = 0; e < N; ++e) {
                 if (!((keepbits >> (e >> 5)) & 1u)) continue;
                 const float sv = row[e];
-                const float key = __fadd_rn(sv, bias_s[e]);
+                const float key = __fadd_rn(sv, bias_t[(e & 31) * S + (e >> 5)]);
                 if (key >= th) top.offer(key, e, sv);
             }
             top.write(K, renorm, route_scale, topk_idx + t * K, topk_w + t * K);
