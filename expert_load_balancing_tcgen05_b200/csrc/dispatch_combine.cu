@@ -21,6 +21,10 @@ namespace moe {
 
 constexpr int DC_THREADS = 256;
 constexpr int DC_WARPS = DC_THREADS / 32;
+// combine runs 4-warp blocks: finer blocks spread its warps evenly over the SMs
+// (at 4096 tokens, 8-warp blocks land 3 or 4 per SM)
+constexpr int CB_THREADS = 128;
+constexpr int CB_WARPS = CB_THREADS / 32;
 
 __device__ __forceinline__ void ld_vec(const void* p, uint4& v) {
     v = __ldg(reinterpret_cast<const uint4*>(p));
@@ -144,16 +148,16 @@ __global__ void __launch_bounds__(DC_THREADS) dispatch_kernel(
 }
 
 template <int EPV>
-__global__ void __launch_bounds__(DC_THREADS) combine_kernel(const char* __restrict__ y, int64_t T, int d,
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const char* __restrict__ y, int64_t T, int d,
                                                              int K, const int32_t* __restrict__ pos,
                                                              const float* __restrict__ w,
                                                              char* __restrict__ out) {
-    __shared__ int s_pos[DC_WARPS][32];
-    __shared__ float s_w[DC_WARPS][32];
+    __shared__ int s_pos[CB_WARPS][32];
+    __shared__ float s_w[CB_WARPS][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row_bytes = (int64_t)d * (16 / EPV);
     const int nvec = d / EPV;
-    for (int64_t t = (int64_t)blockIdx.x * DC_WARPS + warp; t < T; t += (int64_t)gridDim.x * DC_WARPS) {
+    for (int64_t t = (int64_t)blockIdx.x * CB_WARPS + warp; t < T; t += (int64_t)gridDim.x * CB_WARPS) {
         int my_pos = -1;
         float my_w = 0.f;
         if (lane < K) {
@@ -230,8 +234,9 @@ __global__ void __launch_bounds__(DC_THREADS) combine_kernel(const char* __restr
     }
 }
 
-static unsigned dc_blocks(int64_t T) {
-    long long b = (T + DC_WARPS - 1) / DC_WARPS;
+// one warp per token; grid capped at 64 blocks per SM (grid-stride beyond)
+static unsigned token_blocks(int64_t T, int warps_per_block) {
+    long long b = (T + warps_per_block - 1) / warps_per_block;
     const long long cap = (long long)moe_host::sm_count() * 64;
     if (b > cap) b = cap;
     if (b < 1) b = 1;
@@ -241,7 +246,7 @@ static unsigned dc_blocks(int64_t T) {
 cudaError_t launch_dispatch(const void* x, int dtype, int64_t T, int d, int K, const int32_t* slot_idx,
                             const int32_t* offsets, const int32_t* rank, void* rows, uint8_t* rows_fp8,
                             float* scales, int32_t* pos, int32_t* row_src, cudaStream_t st) {
-    const unsigned nb = dc_blocks(T);
+    const unsigned nb = token_blocks(T, DC_WARPS);
     const char* xc = static_cast<const char*>(x);
     char* rc = static_cast<char*>(rows);
     const bool fp8 = rows_fp8 != nullptr;
@@ -263,12 +268,12 @@ cudaError_t launch_dispatch(const void* x, int dtype, int64_t T, int d, int K, c
 
 cudaError_t launch_combine(const void* y, int dtype, int64_t T, int d, int K, const int32_t* pos,
                            const float* w, void* out, cudaStream_t st) {
-    const unsigned nb = dc_blocks(T);
+    const unsigned nb = token_blocks(T, CB_WARPS);
     if (dtype == MOE_BF16)
-        combine_kernel<8><<<nb, DC_THREADS, 0, st>>>(static_cast<const char*>(y), T, d, K, pos, w,
+        combine_kernel<8><<<nb, CB_THREADS, 0, st>>>(static_cast<const char*>(y), T, d, K, pos, w,
                                                      static_cast<char*>(out));
     else
-        combine_kernel<4><<<nb, DC_THREADS, 0, st>>>(static_cast<const char*>(y), T, d, K, pos, w,
+        combine_kernel<4><<<nb, CB_THREADS, 0, st>>>(static_cast<const char*>(y), T, d, K, pos, w,
                                                      static_cast<char*>(out));
     moe_host::note_launch();
     return cudaGetLastError();
