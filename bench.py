@@ -61,7 +61,7 @@ def workload_config(wl):
     return {"workload": f"{wl.name}: T={wl.T} d={wl.d} N={wl.N} K={wl.K} sigmoid, {wl.n_groups} groups keep "
                         f"{wl.topk_groups}, group score top-{wl.group_topn} sum, bias U(-0.01,0.01), "
                         f"weights x{wl.scale}, bf16 x~N(0,1) W~N(0,1/d)",
-            "T": wl.T, "d": wl.d, "N": wl.N, "K": wl.K, "global_batch": None,
+            "T": wl.T, "d": wl.d, "N": wl.N, "K": wl.K,
             "l2": "inputs larger than L2 (x 235 MB, dispatch buffer 1.88 GB per rank); consecutive steps "
                   "alternate between two distinct token batches; no flush"}
 
