@@ -141,3 +141,20 @@ def test_every_call_accepts_an_empty_batch():
     assert L.moe_combine(None, 1, 0, d, K, None, None, None, None) == 0
     assert L.moe_route_balanced(0, K, N, 1.0, None, None, None) == 0
     del e_f
+
+
+@pytest.mark.parametrize("N,K,G,TG,fn", [(512, 8, 16, 4, 1), (32, 4, 4, 2, 1), (512, 16, 1, 1, 0), (16, 3, 1, 1, 0)])
+def test_route_with_gate_outside_the_tensor_core_shapes(orc, N, K, G, TG, fn):
+    # bf16 inputs whose N has no tensor-core tile run the CUDA-core gate, then the general selection kernel
+    T, d = 333, 256
+    wl = W.Workload("edge_gate", 0, T, d, N, K, fn, n_groups=G, topk_groups=TG, group_topn=2, renorm=True,
+                    scale=2.5, has_bias=True)
+    inp = W.make_inputs(wl, seed=N + K)
+    s, idx, w, ws = route_gpu(wl, inp["x"].cuda(), inp["W"].cuda(), None, inp["bias"].cuda())
+    assert lib().moe_workspace_status(ws) == 0
+    h = orc.logits(inp["x"].float().numpy(), inp["W"].float().numpy())
+    s_ref = orc.scores(h, fn)
+    err = np.abs(to_np(s).astype(np.float64) - s_ref)
+    assert (err <= 1e-3 * np.abs(s_ref) + 1e-7).all()
+    ri, rw = orc.select(to_np(s), inp["bias"].numpy(), K, G, TG, 2, True, 2.5)
+    assert np.array_equal(to_np(idx), ri) and np.array_equal(to_np(w), rw)
