@@ -101,7 +101,7 @@ __device__ __forceinline__ int ld_volatile(const int32_t* p) { return *reinterpr
 __device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, int64_t A, int32_t* __restrict__ counts,
                                               int32_t* __restrict__ offsets, moe_stats* stats,
                                               const double* __restrict__ hs_partial, int hs_blocks, int N, int64_t T,
-                                              const ScanCtl* ctl, int* s_scan, double* s_red) {
+                                              const ScanCtl* ctl, int* s_scan, double* s_red, int* s_cnt) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int c8[LS_SLOTS_PER_THREAD];
 #pragma unroll
@@ -120,19 +120,20 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, i
         if (e < n_slots) {
             offsets[e] = run;
             counts[e] = c8[j];
+            s_cnt[e] = c8[j];
         }
         run += c8[j];
     }
     if (tid == 0) offsets[n_slots] = total_i;  // T*K less the dropped assignments
     if (stats == nullptr) return;
+    __syncthreads();  // s_cnt complete
     const double total = (double)total_i;
     const double mean = n_slots > 0 ? total / (double)n_slots : 0.0;
     double mx = 0.0, var = 0.0, H = 0.0, Hs = 0.0;
-#pragma unroll
-    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
-        const int e = tid * LS_SLOTS_PER_THREAD + j;
-        if (e < n_slots) {
-            const double c = (double)c8[j];
+    // one slot per thread (strided), so the fp64 log2 work is spread over the block
+    for (int e = tid; e < n_slots; e += LS_THREADS) {
+        {
+            const double c = (double)s_cnt[e];
             mx = fmax(mx, c);
             var += (c - mean) * (c - mean);
             if (c > 0.0) {
@@ -366,8 +367,9 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
     //    control words for the next call
     if (b == nblk - 1 && counts != nullptr) {  // (the bounded-wait self-test passes no outputs)
         __syncthreads();
+        // the warp histograms are no longer needed: they hold the counts for the statistics
         finish_totals(pre + b * n_slots, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T, ctl,
-                      s_scan, s_red);
+                      s_scan, s_red, wh);
     }
     __syncthreads();
     if (tid == 0) {
