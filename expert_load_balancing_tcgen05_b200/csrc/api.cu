@@ -168,13 +168,22 @@ size_t moe_capacity_workspace_bytes(int64_t T, int32_t K, int32_t N) {
     return capacity_workspace_bytes(T, K, N);
 }
 
+// ceil(1.25 * T*K/N) = ceil(5*T*K / (4*N)), exact in integers (T*K < 2^31
+// for every routed problem, so 5*T*K fits easily in 64 bits)
+int64_t moe_capacity_limit(int64_t T, int32_t K, int32_t N) {
+    if (T < 0 || K <= 0 || N <= 0) return -1;
+    const int64_t num = 5 * T * (int64_t)K, den = 4 * (int64_t)N;
+    return (num + den - 1) / den;
+}
+
 moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, const float* bias, int64_t capacity,
                               int32_t* topk_idx, float* topk_w, moe_capacity_info* info, void* ws,
                               size_t ws_bytes, moe_stream_t stream) {
     moe_status s = check_route_cfg(cfg);
     if (s != MOE_OK) return s;
     const moe_route_cfg& c = *cfg;
-    if (c.K > 16 || capacity < 0) return MOE_ERR_INVALID;
+    if (c.K > 16) return MOE_ERR_INVALID;
+    if (capacity < 0) capacity = moe_capacity_limit(c.T, c.K, c.N);  // the page's 1.25 factor
     if (c.T > 0 && (scores == nullptr || topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID;
     if (scores != nullptr && !aligned16(scores)) return MOE_ERR_INVALID;
     if (ws == nullptr || ws_bytes < moe_capacity_workspace_bytes(c.T, c.K, c.N)) return MOE_ERR_INVALID;
@@ -269,7 +278,7 @@ moe_status moe_workspace_status(void* ws, moe_stream_t stream) {
     const int32_t scan = w.c.sticky | w.c.err;
     moe_status r = MOE_OK;
     if ((w.h.gate_err & 1) || (scan & 1)) r = MOE_ERR_TIMEOUT;
-    else if (scan & 2) r = MOE_ERR_INVALID;
+    else if (scan & 6) r = MOE_ERR_INVALID;  // an expert id out of range, or overlapping calls on one workspace
     if (w.h.gate_err || w.c.sticky) {
         const int32_t z = 0;
         char* base = static_cast<char*>(ws);

@@ -43,7 +43,8 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 struct ScanCtl {
     uint32_t ticket;        // next block index to hand out
     uint32_t done;          // blocks finished
-    int32_t err;            // this call: bit 0 look-back wait ran out; bit 1 expert id out of range
+    int32_t err;            // this call: bit 0 look-back wait ran out; bit 1 expert id out of range;
+                            // bit 2 a ticket past the grid (control words left set by an overlapping call)
     int32_t sticky;         // all calls since the last moe_workspace_status
     uint32_t epoch;         // calls completed; tags this call's look-back flags
     int32_t pad[11];

@@ -186,6 +186,22 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, i
 
 constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
 
+// Block end: the last block to finish folds this call's error bits into the
+// sticky word and resets the control words for the next call.
+__device__ __forceinline__ void block_done(ScanCtl* ctl, int64_t nblk) {
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1)) {
+            __threadfence();
+            ctl->sticky |= ctl->err;
+            ctl->err = 0;
+            ctl->done = 0;
+            ctl->ticket = 0;
+            ctl->epoch = ctl->epoch + 1;
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t flag_tag(uint32_t epoch) { return 0x80000000u | ((epoch & 0x1FFFFFFFu) << 2); }
 // state of a flag word for the call tagged `tag`: 0 unless the word carries the tag
 __device__ __forceinline__ uint32_t flag_state(uint32_t f, uint32_t tag) { return (f & ~3u) == tag ? (f & 3u) : 0u; }
@@ -212,6 +228,13 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
     __syncthreads();
     const int64_t b = s_b;
     const uint32_t tag = s_tag;
+    if (b >= nblk) {
+        // a ticket past the grid: the control words were not reset (two calls
+        // overlapped on one workspace).  Write nothing; report it (bit 2).
+        if (tid == 0) atomicOr(&ctl->err, 4);
+        block_done(ctl, nblk);
+        return;
+    }
 
     // 1. slots, warp histograms, in-warp stable ranks (all loads issued first)
     int32_t* my = wh + warp * n_slots;
@@ -372,17 +395,7 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
                       s_scan, s_red, wh);
     }
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1)) {
-            __threadfence();
-            ctl->sticky |= ctl->err;
-            ctl->err = 0;
-            ctl->done = 0;
-            ctl->ticket = 0;
-            ctl->epoch = ctl->epoch + 1;
-        }
-    }
+    block_done(ctl, nblk);
 }
 
 // ---------------------------------------------------------------------------

@@ -12,10 +12,15 @@
 // library holds MOE_NOALLOC_SCRATCH_BYTES of it until the process exits.  In
 // host code its name is only a host-side stand-in, so the device address is
 // taken with cudaGetSymbolAddress once per device (with that device current)
-// and cached.  All calls share the array and it keeps the last call's
-// contents: the kernels clear what must start at zero (the scan's tile
-// ticket, status words and error word) at the start of every call, and two
-// calls whose kernels overlap on the GPU race on it.
+// and cached for the life of the process (a cudaDeviceReset reloads the
+// module at a new address; the cache is not refreshed).  All calls share the
+// array and it keeps the last call's contents.  The load-statistics kernel
+// leaves its control words (tile ticket, finished-block count, error words,
+// call epoch) reset when its last block finishes, but a call must not depend
+// on the previous one having ended cleanly, so every call here first clears,
+// on its own stream, the control block and the look-back flags of its
+// layout (a few KB).  Two calls whose kernels overlap on the GPU race on the
+// array; the caller must serialise them.
 #include <mutex>
 
 #include "common.cuh"
@@ -66,8 +71,12 @@ extern "C" moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T,
     if (moe_workspace_bytes(T, K, N, n_slots) > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // control block and look-back flags start at zero (the epoch restarts at
+    // 0, and the zeroed flags carry no tag of it)
+    const moe::WsLayout L = moe::ws_layout(T, K, N, n_slots);
+    if (cudaMemsetAsync(static_cast<char*>(ws) + L.ctl, 0, L.ctl_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
     const cudaError_t e = moe::launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets,
-                                                 rank, scores, score_fn, stats, ws,
-                                                 reinterpret_cast<cudaStream_t>(stream));
+                                                 rank, scores, score_fn, stats, ws, st);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -29,7 +29,7 @@ MOE_F32, MOE_BF16 = 0, 1
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
            "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout", "moe_route_balanced",
-           "moe_bias_update_ema", "moe_route_capacity", "moe_capacity_workspace_bytes")
+           "moe_bias_update_ema", "moe_route_capacity", "moe_capacity_workspace_bytes", "moe_capacity_limit")
 
 
 class RouteCfg(ctypes.Structure):
@@ -143,10 +143,15 @@ _lib.moe_route_capacity.argtypes = [ctypes.POINTER(RouteCfg), _P, _P, _I64, _P, 
 _lib.moe_route_capacity.restype = _I32
 
 
+_lib.moe_capacity_limit.argtypes = [_I64, _I32, _I32]
+_lib.moe_capacity_limit.restype = _I64
+
+
 def capacity_limit(T, K, N):
-    """ceil(1.25 * T*K/N): the per-expert token capacity of the "Production
-    Testing" section of the entropy page, in integers."""
-    return (5 * T * K + 4 * N - 1) // (4 * N)
+    """The library's per-expert token capacity, ceil(1.25 * T*K/N) (the
+    "Production Testing" section of the entropy page); moe_route_capacity
+    applies the same rule when given a negative capacity."""
+    return int(_lib.moe_capacity_limit(T, K, N))
 
 
 def capacity_workspace(T, K, N, device="cuda"):

@@ -175,7 +175,8 @@ moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale
  *   3. Weights as in moe_route, over the token's kept slots in k order.
  * scores [T,N] fp32 (moe_route's scores), bias [N] fp32 or NULL; cfg gives T,
  * N, K (<= 16), the groups, renorm and route_scale (d, score_fn, in_dtype are
- * not used).  capacity >= 0 (ceil(1.25*T*K/N) for the page's rule).
+ * not used).  capacity >= 0 sets the per-expert limit; capacity < 0 takes
+ * the page's rule, moe_capacity_limit(T, K, N) = ceil(1.25 * T*K/N).
  * topk_idx, topk_w [T,K] out; info (device, may be NULL) receives the
  * capacity and the overflow / reroute / drop counts.  ws: a zero-filled
  * workspace of moe_capacity_workspace_bytes() bytes, kept between calls.
@@ -191,6 +192,12 @@ typedef struct moe_capacity_info {
 } moe_capacity_info;
 
 size_t moe_capacity_workspace_bytes(int64_t T, int32_t K, int32_t N);
+
+/* The per-expert token capacity of [ENT] "Production Testing": a capacity
+ * factor of 1.25 over the balanced load, ceil(1.25 * T*K / N), computed
+ * exactly in integers as ceil(5*T*K / (4*N)).  Returns -1 for T < 0, K <= 0
+ * or N <= 0. */
+int64_t moe_capacity_limit(int64_t T, int32_t K, int32_t N);
 
 moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, const float* bias,
                               int64_t capacity, int32_t* topk_idx, float* topk_w,
@@ -315,14 +322,18 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
  *  - Returns MOE_ERR_UNSUPPORTED, enqueuing nothing, when the problem needs
  *    more scratch than that (moe_workspace_bytes(T, K, N, n_slots) larger
  *    than MOE_NOALLOC_SCRATCH_BYTES, 4 MiB; the largest routing workload
- *    here, T = 131072 tokens, K = 8, 288 slots, needs about 1.1 MB).
+ *    here, T = 131072 tokens, K = 8, 288 slots, needs 1,706,496 bytes).
  *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
- *  - All calls share the one array, which keeps the last call's contents
- *    (every call re-initialises what it needs).  Calls whose kernels overlap
- *    on the GPU -- different streams, or threads, using the same device --
- *    race on it and must be serialised by the caller.
+ *    that device current) and caches it for the life of the process; make
+ *    that first call before any stream capture.  The cached address does
+ *    not survive cudaDeviceReset (the library's device module is reloaded
+ *    at a new address): do not call this entry point after a device reset.
+ *  - All calls share the one array, which keeps the last call's contents.
+ *    Every call first clears, on its stream, the part that must start at
+ *    zero (the scan's control words and look-back flags, a few KB), so a
+ *    call never depends on how the previous one ended.  Calls whose kernels
+ *    overlap on the GPU -- different streams, or threads, using the same
+ *    device -- race on the array: the caller must serialise them.
  * The load status of the call is in stats->status, as for moe_load_stats.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -334,7 +345,8 @@ moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T, int32_t K,
 
 /* Synchronises `stream`, reads and clears the workspace's sticky device
  * error words: MOE_OK, MOE_ERR_TIMEOUT if a bounded wait ran out, or
- * MOE_ERR_INVALID if an expert id was out of range, since the last check.
+ * MOE_ERR_INVALID if an expert id was out of range or two load-statistics
+ * calls overlapped on the workspace, since the last check.
  * (The calls that synchronise are this one and moe_selftest_wait_timeout.) */
 moe_status moe_workspace_status(void* ws, moe_stream_t stream);
 

@@ -112,7 +112,8 @@ def test_route_capacity_rejects_bad_arguments(moe):
     ws = L.moe_capacity_workspace_bytes(64, 8, 256)
     assert ws > L.moe_workspace_bytes(64, 8, 256, 256)
     cfg = _cfg(moe)
-    assert L.moe_route_capacity(ctypes.byref(cfg), FAKE, None, -1, FAKE, FAKE, None, FAKE, ws, None) == 1
+    # a negative capacity selects the page's rule; the missing scores are still rejected before any launch
+    assert L.moe_route_capacity(ctypes.byref(cfg), None, None, -1, FAKE, FAKE, None, FAKE, ws, None) == 1
     assert L.moe_route_capacity(ctypes.byref(_cfg(moe, K=17, n_groups=1)), FAKE, None, 5, FAKE, FAKE, None, FAKE,
                                 ws, None) == 1
     assert L.moe_route_capacity(ctypes.byref(cfg), None, None, 5, FAKE, FAKE, None, FAKE, ws, None) == 1
@@ -159,3 +160,16 @@ def test_binding_refuses_cpu_tensors(moe):
     import torch
     with pytest.raises(ValueError):
         moe._ptr(torch.zeros(4))
+
+
+def test_capacity_limit_is_the_pages_rule(moe):
+    """moe_capacity_limit computes ceil(1.25*T*K/N) in the library (the entropy
+    page's "Production Testing" capacity factor), equal to the pinned oracle rule."""
+    import oracle
+    L = moe._lib
+    for T, K, N in ((16384, 8, 256), (4096, 8, 256), (131072, 8, 256), (65536, 8, 128), (512, 2, 8), (6, 1, 4),
+                    (3, 2, 4), (7, 1, 4), (0, 8, 256), (1, 1, 1000), (1 << 27, 8, 2048)):
+        assert L.moe_capacity_limit(T, K, N) == oracle.capacity_limit(T, K, N), (T, K, N)
+        assert moe.capacity_limit(T, K, N) == oracle.capacity_limit(T, K, N)
+    assert L.moe_capacity_limit(-1, 8, 256) == -1 and L.moe_capacity_limit(16, 0, 256) == -1
+    assert L.moe_capacity_limit(16, 8, 0) == -1

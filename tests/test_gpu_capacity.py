@@ -151,3 +151,18 @@ def test_dropped_assignments_through_dispatch_and_combine(orc):
     ref = orc.combine(rows.float().cpu().numpy(), pos_ref, to_np(w))
     got = to_np(out).astype(np.float64)
     assert (np.abs(got - ref) <= np.maximum(2e-2, np.abs(ref) * 2.0 ** -8)).all()
+
+
+@pytest.mark.parametrize("name", ["v3_router", "metric"])
+def test_negative_capacity_is_the_pages_rule(orc, name):
+    """capacity < 0: the library applies ceil(1.25*T*K/N) itself (entropy page,
+    "Production Testing"); the result equals the oracle run at that capacity."""
+    wl = W.WORKLOADS[name]
+    s, b = _gpu_scores(wl, seed=17)
+    idx, w, info, _ = _capacity_gpu(wl, s, b, -1)
+    C = orc.capacity_limit(wl.T, wl.K, wl.N)
+    assert info["capacity"] == C
+    ri, rw, rinfo = orc.route_capacity(to_np(s), to_np(b), wl.K, wl.n_groups, wl.topk_groups, wl.group_topn,
+                                       wl.renorm, wl.scale, capacity=C)
+    assert np.array_equal(to_np(idx), ri) and np.array_equal(to_np(w), rw)
+    assert info == rinfo
