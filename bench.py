@@ -591,6 +591,301 @@ def run_kernel_report():
     print(f"\nbounds: HBM {hbm} GB/s (measured copy), bf16 {tf_burst} TFLOP/s (measured burst)")
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_pipeline(wl, n, threads=None):
+    """The oracle (as it stands) on the first n tokens of a workload: the
+    stage set of the GPU pipeline -- fp64 gate, scores, selection,
+    histogram/positions, stats, bias step, dispatch rows (+ the replica plan
+    and the remap over the replica slots, + the FP8 copy, where the workload
+    has them).  Returns (seconds, threads used)."""
+    import torch
+    import oracle
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    sw = wl.with_(T=n)
+    inp = W.make_inputs(sw, seed=wl.seed)
+    x = inp["x"].float().numpy()
+    Wg = inp["W"].float().numpy()
+    off = inp["off"].numpy() if inp["off"] is not None else None
+    b = inp["bias"].numpy() if inp["bias"] is not None else None
+    xb = inp["x"].view(torch.int16).numpy() if wl.dtype == torch.bfloat16 else inp["x"].numpy()
+    old = oracle.num_threads()
+    if threads is not None:
+        oracle.set_num_threads(threads)
+    used = oracle.num_threads()
+    try:
+        t0 = time.perf_counter()
+        s = oracle.scores(oracle.logits(x, Wg, off), wl.fn)
+        idx, w = oracle.select(s, b, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+        slot, n_slots = idx, wl.N
+        counts, offsets, pos, rk, src = oracle.positions(idx, wl.N)
+        if wl.n_replicas:
+            rs = oracle.replica_plan(counts, wl.n_replicas)
+            slot, n_slots = oracle.apply_replicas(idx, rs), wl.n_slots
+            counts, offsets, pos, rk, src = oracle.positions(slot, n_slots)
+        oracle.load_stats(counts)
+        if b is not None:
+            oracle.bias_update(counts[:wl.N], n * wl.K, b, 0.001, 0)
+        rows = oracle.dispatch_rows(xb, pos)
+        if wl.fp8:
+            oracle.fp8_rows(oracle.dispatch_rows(x, pos))
+        del rows
+        return time.perf_counter() - t0, used
+    finally:
+        oracle.set_num_threads(old)
+
+
+def _oracle_rate(wl, seconds, threads=None):
+    """tokens/s of the oracle pipeline on a sample sized for about `seconds`."""
+    probe = min(wl.T, 64)
+    tp, _ = _oracle_pipeline(wl, probe, threads)
+    n = int(max(probe, min(wl.T, probe * seconds / max(tp, 1e-4))))
+    dt, used = _oracle_pipeline(wl, n, threads)
+    reps = 1
+    while dt < 0.25 * seconds and n == wl.T:  # the whole workload is quick: repeat it
+        reps *= 2
+        dt = sum(_oracle_pipeline(wl, n, threads)[0] for _ in range(reps))
+    return n * reps / dt, (f"{n} tokens" + (f" x {reps}" if reps > 1 else "")), dt, used
+
+
+def run_report(oracle_seconds: float = 4.0):
+    """Three markdown sections, each GPU number produced through the library's
+    C ABI and checked in the same run against the oracle:
+    1. the collapse workload's 100 sign-rule bias steps on fixed scores: per
+       step std/mean, max/mean and load entropy from moe_stats;
+    2. the prefill workload's per-slot loads and imbalance before and after
+       the 32 replicas;
+    3. per workload, the GPU pipeline (route, load statistics, bias step,
+       dispatch) in routed tokens/s and GB/s against its roofline, beside the
+       oracle on the host cores (all cores; one core for the two smallest
+       workloads) on a bounded sample."""
+    import numpy as np
+    import torch
+    import oracle
+    from expert_load_balancing_tcgen05_b200 import moe
+    from expert_load_balancing_tcgen05_b200 import workloads as W
+    hbm, tf_burst, _, peak_kind = _peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    out = []
+    P = out.append
+
+    def route_scores(wl, inp, T=None):
+        T = wl.T if T is None else T
+        scores = torch.empty(T, wl.N, device=dev)
+        idx = torch.empty(T, wl.K, dtype=torch.int32, device=dev)
+        w = torch.empty(T, wl.K, device=dev)
+        ws = moe.workspace(T, wl.K, wl.N, wl.n_slots, device=dev)
+        cfg = moe.route_cfg(T, wl.d, wl.N, wl.K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm,
+                            wl.scale, moe.MOE_BF16 if wl.dtype == torch.bfloat16 else moe.MOE_F32)
+        moe.moe_route(cfg, inp["x"], inp["W"], inp["off"], inp["bias"], scores, idx, w, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_workspace_status(ws) == moe.MOE_OK
+        return cfg, scores, idx, w, ws
+
+    def stats_match(st, ref):
+        ok = st["status"] == 0 and st["total"] == int(ref["total"]) and st["max_load"] == int(ref["max"])
+        for g in ("mean", "imbalance", "std_over_mean", "entropy_load_bits"):
+            ok = ok and abs(st[g] - ref[g]) <= 1e-6 * abs(ref[g]) + 1e-12
+        return ok
+
+    # ---------------------------------------------------------------- 1. collapse
+    wl = W.WORKLOADS["collapse"]
+    T, N, K = wl.T, wl.N, wl.K
+    inp = W.make_inputs(wl, device=dev)
+    cfg, scores, idx, w, ws = route_scores(wl, inp)
+    s_np = scores.cpu().numpy()
+    bias = inp["bias"].clone()
+    b_ref = inp["bias"].cpu().numpy().copy()
+    counts = torch.empty(N, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    rank = torch.empty(T, K, dtype=torch.int32, device=dev)
+    stats = moe.empty_stats(dev)
+    rows_c3 = []
+    all_ok = True
+    for step in range(wl.bias_steps + 1):
+        moe.moe_route(cfg, None, None, None, bias, scores, idx, w, ws)
+        moe.moe_load_stats(idx, T, K, N, None, N, None, counts, offsets, rank, None, wl.fn, stats, ws)
+        if step < wl.bias_steps:
+            moe.moe_bias_update(counts, N, T * K, 0.001, 0, bias)
+        st = moe.read_stats(stats)
+        ri, _ = oracle.select(s_np, b_ref, K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+        c_ref = oracle.histogram(ri, N)
+        ok = bool(np.array_equal(counts.cpu().numpy(), c_ref)) and stats_match(st, oracle.load_stats(c_ref))
+        all_ok = all_ok and ok
+        celeb = int(sum(c_ref[e] for e in W.CELEBRITY_EXPERTS))
+        rows_c3.append((step, st["max_load"], st["imbalance"], st["std_over_mean"], st["entropy_load_bits"], celeb, ok))
+        if step < wl.bias_steps:
+            b_ref = oracle.bias_update(c_ref, T * K, b_ref, 0.001, 0)
+    bias_ok = bool(np.array_equal(bias.cpu().numpy(), b_ref))
+    P(f"## 1. Collapse workload: 100 bias steps (T={T} d={wl.d} N={N} K={K}, sigmoid, 8 groups keep 4, "
+      f"+2.0 logit offset on experts {list(W.CELEBRITY_EXPERTS)}, u = 0.001)\n")
+    P("One gate pass (moe_route, tcgen05), then per step: moe_route from the fixed scores with the current bias "
+      "-> moe_load_stats -> moe_bias_update (sign rule).  Row i is the routing made with the bias after i steps "
+      "(row 100: the final bias).  'oracle' = the GPU counts equal the oracle's replay on the same scores and its "
+      "stats agree within 1e-6.  Mean load = T*K/N = %d.  Monitoring bar of the deployment page: std <= 20%% of "
+      "the mean.\n" % (T * K // N))
+    P("| step | max load | max/mean | std/mean | H_load (bits) | load on the 5 celebrity experts | oracle |")
+    P("|---|---|---|---|---|---|---|")
+    for r in rows_c3:
+        P(f"| {r[0]} | {r[1]} | {r[2]:.4f} | {r[3]:.4f} | {r[4]:.4f} | {r[5]} | {'yes' if r[6] else 'NO'} |")
+    first_ok = next((r[0] for r in rows_c3 if r[3] <= 0.2), None)
+    P(f"\nEvery step matches the oracle: {'yes' if all_ok else 'NO'}; final bias bit-exact: "
+      f"{'yes' if bias_ok else 'NO'}.  log2 N = {np.log2(N):.4f} bits.  First step with std/mean <= 0.20: "
+      f"{first_ok}.\n")
+    del inp, scores, idx, w, ws, rank
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- 2. prefill replicas
+    wl = W.WORKLOADS["prefill_replicas"]
+    T, N, K, R = wl.T, wl.N, wl.K, wl.n_replicas
+    inp = W.make_inputs(wl, device=dev)
+    cfg, scores, idx, w, ws = route_scores(wl, inp)
+    ri, _ = oracle.select(scores.cpu().numpy(), inp["bias"].cpu().numpy(), K, wl.n_groups, wl.topk_groups,
+                          wl.group_topn, wl.renorm, wl.scale)
+    sel_ok = bool(np.array_equal(idx.cpu().numpy(), ri))
+    del scores
+    slot = torch.empty(T, K, dtype=torch.int32, device=dev)
+    rank = torch.empty(T, K, dtype=torch.int32, device=dev)
+    c1 = torch.empty(N, dtype=torch.int32, device=dev)
+    o1 = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    st1 = moe.empty_stats(dev)
+    moe.moe_load_stats(idx, T, K, N, None, N, slot, c1, o1, rank, None, wl.fn, st1, ws)
+    rs = torch.empty(N, dtype=torch.int32, device=dev)
+    moe.moe_replica_plan(c1, N, R, rs)
+    c2 = torch.empty(N + R, dtype=torch.int32, device=dev)
+    o2 = torch.empty(N + R + 1, dtype=torch.int32, device=dev)
+    st2 = moe.empty_stats(dev)
+    moe.moe_load_stats(idx, T, K, N, rs, N + R, slot, c2, o2, rank, None, wl.fn, st2, ws)
+    torch.cuda.synchronize()
+    before, after = moe.read_stats(st1), moe.read_stats(st2)
+    cb, ca, rsn = c1.cpu().numpy(), c2.cpu().numpy(), rs.cpu().numpy()
+    cb_ref = oracle.histogram(ri, N)
+    rs_ref = oracle.replica_plan(cb_ref, R)
+    ca_ref, _, _, rk_ref, _ = oracle.positions(oracle.apply_replicas(ri, rs_ref), N + R)
+    ok5 = (sel_ok and np.array_equal(cb, cb_ref) and np.array_equal(rsn, rs_ref) and np.array_equal(ca, ca_ref)
+           and np.array_equal(rank.cpu().numpy(), rk_ref) and stats_match(before, oracle.load_stats(cb_ref))
+           and stats_match(after, oracle.load_stats(ca_ref)))
+    P(f"## 2. Prefill workload with redundant experts (T={T} d={wl.d} N={N} K={K}, Zipf(1.1) logit offsets "
+      f"-1.1*ln(e+1), {R} replicas -> {N + R} slots)\n")
+    P("moe_route (tcgen05 gate, selection in the epilogue) -> moe_load_stats over the 256 experts -> "
+      "moe_replica_plan (32 hottest by count, ties to the lower index) -> moe_load_stats over the 288 slots (odd "
+      "tokens of a replicated expert go to its replica).  Before replication the 32 replica slots are empty and "
+      "max/mean is taken over the 256 experts (mean T*K/256); after, over the 288 slots (mean T*K/288).\n")
+    P("| | slots | max load | mean | max/mean | std/mean | H_load (bits) |")
+    P("|---|---|---|---|---|---|---|")
+    for name, st in (("before", before), ("after", after)):
+        P(f"| {name} | {st['n_slots']} | {st['max_load']} | {st['mean']:.2f} | {st['imbalance']:.4f} | "
+          f"{st['std_over_mean']:.4f} | {st['entropy_load_bits']:.4f} |")
+    P(f"\nGPU selection, histograms, replica plan, slot counts, ranks and stats equal the oracle's (on the GPU's "
+      f"scores): {'yes' if ok5 else 'NO'}.\n")
+    P("Per-slot loads (slot: before -> after; slots 256.. are the replicas, with the expert they copy):\n")
+    P("| slot | expert | before | after |")
+    P("|---|---|---|---|")
+    owner = {int(rsn[e]): e for e in range(N) if rsn[e] >= 0}
+    for sl in range(N + R):
+        e = sl if sl < N else owner.get(sl, -1)
+        P(f"| {sl} | {e} | {int(cb[sl]) if sl < N else 0} | {int(ca[sl])} |")
+    P("")
+    del inp, idx, w, ws, slot, rank
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- 3. per workload, GPU beside the oracle
+    def t_us(fn, n=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / n * 1e3
+
+    P("## 3. Routed tokens/s per workload: the GPU pipeline beside the oracle\n")
+    P(f"GPU: route (gate + selection) -> load statistics (+ replica plan and the slot remap for the prefill "
+      f"workload) -> bias step (workloads with a bias) -> dispatch (+ FP8 copy for the softmax-dispatch "
+      f"workload), one stream, 10 pipelines captured in a CUDA graph and replayed under CUDA events.  Roofline = "
+      f"sum over the stages of max(bytes / {hbm:.1f} GB/s, gate flops / {tf_burst:.1f} TFLOP/s) ({peak_kind} "
+      f"peaks).  Oracle: the same stage set in plain C (fp64), on a bounded sample of each workload's tokens, on "
+      f"the host: CPU '{_cpu_model()}', {os.cpu_count()} logical CPUs.\n")
+    P("| workload | shape | GPU us/batch | GPU routed tokens/s | GPU GB/s (algorithmic) | fraction of roofline | "
+      "oracle tokens/s (threads) | oracle sample | oracle 1 thread tokens/s | GPU / oracle |")
+    P("|---|---|---|---|---|---|---|---|---|---|")
+    for name in ("tiny_softmax", "v3_router", "collapse", "softmax_dispatch", "prefill_replicas", "metric"):
+        wl = W.WORKLOADS[name]
+        T, d, N, K = wl.T, wl.d, wl.N, wl.K
+        A = T * K
+        es = 2 if wl.dtype == torch.bfloat16 else 4
+        inp = W.make_inputs(wl, device=dev, seed=wl.seed)
+        x, Wg, off, bias = inp["x"], inp["W"], inp["off"], inp["bias"]
+        scores = torch.empty(T, N, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        w = torch.empty(T, K, device=dev)
+        ws = moe.workspace(T, K, N, wl.n_slots, device=dev)
+        cfg = moe.route_cfg(T, d, N, K, wl.fn, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale,
+                            moe.MOE_BF16 if wl.dtype == torch.bfloat16 else moe.MOE_F32)
+        slot = torch.empty(T, K, dtype=torch.int32, device=dev)
+        rank = torch.empty(T, K, dtype=torch.int32, device=dev)
+        counts = torch.empty(wl.n_slots, dtype=torch.int32, device=dev)
+        offsets = torch.empty(wl.n_slots + 1, dtype=torch.int32, device=dev)
+        stats = moe.empty_stats(dev)
+        rs = torch.empty(N, dtype=torch.int32, device=dev) if wl.n_replicas else None
+        b2 = bias.clone() if bias is not None else None
+        rows = torch.empty(A, d, dtype=wl.dtype, device=dev)
+        q = torch.empty(A, d, dtype=torch.uint8, device=dev) if wl.fp8 else None
+        sc = torch.empty(A, d // 128, device=dev) if wl.fp8 else None
+        pos = torch.empty(T, K, dtype=torch.int32, device=dev)
+
+        def pipeline():
+            moe.moe_route(cfg, x, Wg, off, b2, scores, idx, w, ws)
+            if rs is not None:
+                moe.moe_load_stats(idx, T, K, N, None, N, slot, counts[:N], offsets[:N + 1], rank, None, wl.fn,
+                                   stats, ws)
+                moe.moe_replica_plan(counts[:N], N, wl.n_replicas, rs)
+            moe.moe_load_stats(idx, T, K, N, rs, wl.n_slots, slot, counts, offsets, rank, None, wl.fn, stats, ws)
+            if b2 is not None:
+                moe.moe_bias_update(counts[:N], N, A, 0.001, 0, b2)
+            moe.moe_dispatch(x, T, d, K, slot, offsets, rank, rows, q, sc, pos, None)
+
+        us = t_us(pipeline)
+        nbytes = (T * d * es + N * d * es + T * N * 4 + A * 8) + (T * N * 4 + A * 8) + A * 12 + \
+            (T * d * es + A * d * es + A * 12) + ((A * d + A * d // 32) if wl.fp8 else 0)
+        # serial roofline: the gate at the slower of its HBM and tensor bounds, the rest at HBM speed
+        gate_b = T * d * es + N * d * es + T * N * 4
+        roof = (max(gate_b / (hbm * 1e9), 2 * T * d * N / (tf_burst * 1e12)) + (nbytes - gate_b) / (hbm * 1e9)) * 1e6
+        gpu_tps = T / (us / 1e6)
+        del inp, x, Wg, scores, idx, w, ws, slot, rank, rows, q, sc, pos
+        torch.cuda.empty_cache()
+        o_tps, n, dt, used = _oracle_rate(wl, oracle_seconds)
+        one = ""
+        if name in ("tiny_softmax", "v3_router"):
+            o1, n1, dt1, _ = _oracle_rate(wl, oracle_seconds, threads=1)
+            one = f"{o1:,.0f} ({n1}, {dt1:.1f} s)"
+        P(f"| {name} | T={T} d={d} N={N} K={K} | {us:.1f} | {gpu_tps:,.0f} | {nbytes / (us / 1e6) / 1e9:,.0f} | "
+          f"{roof / us:.2f} | {o_tps:,.0f} ({used}) | {n}, {dt:.1f} s | {one or '-'} | "
+          f"{gpu_tps / o_tps:,.0f} |")
+    P("")
+    print("\n".join(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,6 +895,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels", action="store_true",
                     help="print per-call device times of every workload against their bounds (markdown)")
+    ap.add_argument("--report", action="store_true",
+                    help="print the bias-balancing trajectory, the replica loads and per-workload GPU vs oracle "
+                         "throughput (markdown)")
     ap.add_argument("--serial", action="store_true",
                     help="time the serial schedule (one call after another) instead of the pipelined one")
     args = ap.parse_args()
@@ -612,6 +910,9 @@ def main():
 
     if args.kernels:
         run_kernel_report()
+        return
+    if args.report:
+        run_report()
         return
     if args.impl == "reference":
         if rank == 0:
