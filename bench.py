@@ -131,7 +131,7 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------
-def make_step(wl, rank, dev, world, pipelined):
+def make_step(wl, rank, dev, world, pipelined, fused=False):
     """The routing step on this rank's batches (inputs drawn on the device).
     Consecutive steps alternate between two distinct token batches in
     different buffers, so that overlapped steps never share rows of x in L2."""
@@ -140,7 +140,7 @@ def make_step(wl, rank, dev, world, pipelined):
     inp = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank)
     x2 = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank + 50)["x"]
     return RoutingStep(wl, [inp["x"], x2], inp["W"], inp["bias"].clone(), inp["off"], dev, world=world,
-                       pipelined=pipelined)
+                       pipelined=pipelined, fused=fused)
 
 
 def stage_bytes(wl):
@@ -202,7 +202,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[WORKLOAD_NAME]
     pipelined = not args.serial
-    P = make_step(wl, rank, dev, world, pipelined)
+    P = make_step(wl, rank, dev, world, pipelined, fused=args.fused)
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
 
     def barrier():
@@ -258,7 +258,7 @@ def run_ours(args, rank, world, local_rank):
 
     # the serial schedule: per-stage times (route, load statistics + bias
     # step, dispatch), the combine loop and the end-to-end leg
-    S = make_step(wl, rank, dev, world, pipelined=False)
+    S = make_step(wl, rank, dev, world, pipelined=False, fused=args.fused)
     for _ in range(3):
         S.step()
     n_stage = max(3, min(args.steps, 50))
@@ -302,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     # the device for the expert GEMMs.
     del S
     torch.cuda.empty_cache()
-    E2 = make_step(wl, rank, dev, world, pipelined)
+    E2 = make_step(wl, rank, dev, world, pipelined, fused=args.fused)
     x_host = E2.x.cpu().pin_memory()
     x_dev = [torch.empty_like(E2.x) for _ in range(2)]
     res_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in E2.results(E2.sets[0])]
@@ -353,6 +353,9 @@ def run_ours(args, rank, world, local_rank):
         schedule = ("pipelined: the routing of batch i+1 (gate on "
                     f"{PIPELINED_GATE_CTAS} SMs, selection, load statistics, bias step) on a high-priority stream beside "
                     "the dispatch of batch i") if pipelined else "serial: one call after another on one stream"
+        schedule += ("; routing through the fused path (selection and per-tile histograms in the gate's epilogue, "
+                     "no scores in memory; statistics from the tile histograms)") if args.fused else \
+            "; routing through the gate's scores epilogue and the selection kernel"
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -473,7 +476,7 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def run_kernel_report():
+def run_kernel_report(only=None):
     """Per-call device times of the library on every workload (3 warm-up
     calls, then 10 calls captured in a CUDA graph and replayed under CUDA
     events), each against its bound: HBM
@@ -513,7 +516,10 @@ def run_kernel_report():
         bound = max(nbytes / (hbm * 1e9), flops / (tf_burst * 1e12)) * 1e6
         rows.append((wl.name, f"T={wl.T} d={wl.d} N={wl.N} K={wl.K}", call, us, bound, bound / us, note))
 
-    for name in ("tiny_softmax", "v3_router", "collapse", "softmax_dispatch", "prefill_replicas", "metric"):
+    names = ("tiny_softmax", "v3_router", "collapse", "softmax_dispatch", "prefill_replicas", "metric")
+    for name in names:
+        if only is not None and name != only:
+            continue
         wl = W.WORKLOADS[name]
         T, d, N, K = wl.T, wl.d, wl.N, wl.K
         A = T * K
@@ -532,6 +538,14 @@ def run_kernel_report():
             2 * T * d * N)
         sel = lambda: moe.moe_route(cfg, None, None, None, bias, scores, idx, w, ws)
         add(wl, "  selection alone (scores given)", t_us(sel), T * N * 4 + A * 8)
+        fusable = wl.dtype == torch.bfloat16 and N in (64, 128, 256) and K <= 8 and \
+            (wl.n_groups == 1 or (wl.fn == moe.MOE_SIGMOID and N // wl.n_groups == 32))
+        tiles = None
+        if fusable:
+            tiles = torch.empty(moe.tile_counts_shape(T, N), dtype=torch.int32, device=dev)
+            rt = lambda: moe.moe_route_tiles(cfg, x, Wg, off, bias, idx, w, tiles, ws)
+            add(wl, "moe_route_tiles (gate + selection + tile histograms in the epilogue)", t_us(rt),
+                T * d * es + N * d * es + A * 8 + tiles.numel() * 4, 2 * T * d * N)
         route()
         slot = torch.empty(T, K, dtype=torch.int32, device=dev)
         rank = torch.empty(T, K, dtype=torch.int32, device=dev)
@@ -549,6 +563,12 @@ def run_kernel_report():
         ls = lambda: moe.moe_load_stats(idx, T, K, N, rep, n_slots, slot, counts, offsets, rank, None, wl.fn, stats,
                                         ws)
         add(wl, "moe_load_stats", t_us(ls), A * 12 + n_slots * 8, note="latency-bound (single-pass scan)")
+        if tiles is not None:
+            moe.moe_route_tiles(cfg, x, Wg, off, bias, idx, w, tiles, ws)
+            lst = lambda: moe.moe_load_stats_tiles(idx, T, K, N, tiles, rep, n_slots, slot, counts, offsets, rank,
+                                                   stats, ws)
+            add(wl, "moe_load_stats_tiles", t_us(lst), A * 12 + tiles.numel() * 4 + n_slots * 8,
+                note="latency-bound (single-pass scan)")
         ls()
         if wl.bias_steps or wl.has_bias:
             b2 = bias.clone() if bias is not None else torch.zeros(N, device=dev)
@@ -895,9 +915,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels", action="store_true",
                     help="print per-call device times of every workload against their bounds (markdown)")
+    ap.add_argument("--only", default=None,
+                    help="with --kernels: report one workload only (tiny_softmax, v3_router, collapse, "
+                         "softmax_dispatch, prefill_replicas, metric)")
     ap.add_argument("--report", action="store_true",
                     help="print the bias-balancing trajectory, the replica loads and per-workload GPU vs oracle "
                          "throughput (markdown)")
+    ap.add_argument("--fused", action="store_true",
+                    help="route through the fused path (selection and tile histograms in the gate's epilogue)")
     ap.add_argument("--serial", action="store_true",
                     help="time the serial schedule (one call after another) instead of the pipelined one")
     args = ap.parse_args()
@@ -909,7 +934,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.kernels:
-        run_kernel_report()
+        run_kernel_report(args.only)
         return
     if args.report:
         run_report()

@@ -13,7 +13,7 @@ bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn);
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
                            bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
-                           int max_ctas, cudaStream_t st);
+                           int max_ctas, int32_t* tile_counts, cudaStream_t st);
 cudaError_t launch_gate_simt(const void* x, const void* W, int dtype, const float* off, const float* logit_bias,
                              int T, int d, int N, int fn, float* scores, cudaStream_t st);
 cudaError_t launch_bias_update_ema(const int32_t* counts, int N, int64_t total, float u, float alpha, float* ema,
@@ -28,7 +28,8 @@ cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int
                               float* w, cudaStream_t st);
 cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const int32_t* replica_slot,
                               int n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets, int32_t* rank,
-                              const float* scores, int score_fn, moe_stats* stats, void* ws, cudaStream_t st);
+                              const float* scores, int score_fn, moe_stats* stats, void* ws, cudaStream_t st,
+                              const int32_t* tile_counts = nullptr);
 cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t st);
 cudaError_t launch_replica_plan(const int32_t* counts, int N, int R, int32_t* replica_slot, cudaStream_t st);
 cudaError_t launch_bias_update(const int32_t* counts, int N, int64_t total, float u, int mode, float* bias,
@@ -134,7 +135,8 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
             if (c.d % 8 != 0 || !aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID;
             e = launch_gate_tc(x, w_gate, logit_offset, bias, c.T, c.d, c.N, c.K, c.score_fn, c.n_groups,
                                eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, fused,
-                               bias_in_logits, scores, topk_idx, topk_w, &hdr->gate_err, c.gate_max_ctas, st);
+                               bias_in_logits, scores, topk_idx, topk_w, &hdr->gate_err, c.gate_max_ctas, nullptr,
+                               st);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
             if (fused) return MOE_OK;
         } else {
@@ -145,6 +147,28 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
     }
     return cuda_status(launch_route_topk(scores, sel_bias, c.T, c.N, c.K, c.n_groups, eff_topk_groups,
                                          c.group_topn, c.renorm ? 1 : 0, c.route_scale, topk_idx, topk_w, st));
+}
+
+moe_status moe_route_tiles(const moe_route_cfg* cfg, const void* x, const void* w_gate, const float* logit_offset,
+                           const float* bias, int32_t* topk_idx, float* topk_w, int32_t* tile_counts, void* ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+    moe_status s = check_route_cfg(cfg);
+    if (s != MOE_OK) return s;
+    const moe_route_cfg& c = *cfg;
+    if (x == nullptr || w_gate == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+    if (c.T > 0 && (topk_idx == nullptr || topk_w == nullptr || tile_counts == nullptr)) return MOE_ERR_INVALID;
+    if (c.d <= 0 || c.in_dtype != MOE_BF16) return c.in_dtype == MOE_F32 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID;
+    if (!gate_tc_supported(c.N) || !gate_tc_can_fuse(c.N, c.K, c.score_fn, c.n_groups, c.group_topn))
+        return MOE_ERR_UNSUPPORTED;
+    if (c.d % 8 != 0 || !aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID;
+    if (ws_bytes < moe_workspace_bytes(c.T, c.K, c.N, c.N)) return MOE_ERR_INVALID;
+    if (c.T == 0) return MOE_OK;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(static_cast<char*>(ws) + ws_layout(c.T, c.K, c.N, c.N).header);
+    const int eff_topk_groups = c.n_groups > 1 ? c.topk_groups : 1;
+    return cuda_status(launch_gate_tc(x, w_gate, logit_offset, bias, c.T, c.d, c.N, c.K, c.score_fn, c.n_groups,
+                                      eff_topk_groups, c.group_topn, c.renorm ? 1 : 0, c.route_scale, /*fused=*/true,
+                                      c.bias_mode == 1, nullptr, topk_idx, topk_w, &hdr->gate_err, c.gate_max_ctas,
+                                      tile_counts, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N, const int32_t* replica_slot,
@@ -161,6 +185,21 @@ moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t
     if (ws_bytes < moe_workspace_bytes(T, K, N, n_slots)) return MOE_ERR_INVALID;
     return cuda_status(launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets, rank,
                                          scores, score_fn, stats, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_load_stats_tiles(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
+                                const int32_t* tile_counts, const int32_t* replica_slot, int32_t n_slots,
+                                int32_t* slot_idx, int32_t* counts, int32_t* offsets, int32_t* rank, moe_stats* stats,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (T < 0 || K <= 0 || K > 32 || N <= 0 || n_slots < N || n_slots > MAX_SLOTS) return MOE_ERR_INVALID;
+    if (T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
+    if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+    if (T > 0 && (topk_idx == nullptr || rank == nullptr || tile_counts == nullptr)) return MOE_ERR_INVALID;
+    if (replica_slot == nullptr && n_slots != N) return MOE_ERR_INVALID;
+    if (ws_bytes < moe_workspace_bytes(T, K, N, n_slots)) return MOE_ERR_INVALID;
+    return cuda_status(launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets, rank,
+                                         nullptr, MOE_SIGMOID, stats, ws, reinterpret_cast<cudaStream_t>(stream),
+                                         tile_counts));
 }
 
 size_t moe_capacity_workspace_bytes(int64_t T, int32_t K, int32_t N) {

@@ -27,7 +27,7 @@ cudaError_t launch_capacity_candidates(const float* scores, const float* bias, i
 cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const int32_t* replica_slot,
                               int n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets,
                               int32_t* rank, const float* scores, int score_fn, moe_stats* stats,
-                              void* ws, cudaStream_t st);
+                              void* ws, cudaStream_t st, const int32_t* tile_counts = nullptr);
 
 constexpr int CAP_THREADS = 256;
 constexpr int CAP_KMAX = 16;

@@ -58,6 +58,7 @@ constexpr int LS_BLOCK = LS_WARPS * LS_CHUNKS * 32;  // 2048 assignments per blo
 constexpr int MAX_SLOTS = 2048;                // smem: 8 warps x 2048 x 4 B = 64 KB
 constexpr int LS_SLOTS_PER_THREAD = MAX_SLOTS / LS_THREADS;
 constexpr int HS_BLOCKS = 256;                 // blocks of the score-entropy pass
+constexpr int V2_MAX_BLOCKS = 320;             // largest grid of the chain-free load-statistics kernel
 constexpr int MAX_N = 1024;                    // experts supported by selection / stats
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

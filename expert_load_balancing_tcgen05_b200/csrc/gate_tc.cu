@@ -152,8 +152,9 @@ struct Cfg {
     static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;  // 128, 256 or 512: powers of two
     // epilogue exchange (per token row): 2 x 2 reduction floats, up to 8 group
-    // scores, one 8-entry candidate list (key, score, index)
-    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8) * 4 + 2 * EPI_WARPS * 4;
+    // scores, one 8-entry candidate list (key, score, index); the wait
+    // verdicts; the tile's expert histogram by token parity (2 x BN counts)
+    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8) * 4 + 2 * EPI_WARPS * 4 + 2 * BN * 4;
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
                                          8 * (2 * STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
@@ -166,6 +167,7 @@ struct Epi {
     float* scores;      // [T, N] or null (fused only)
     int32_t* idx;       // [T, K]
     float* w;           // [T, K]
+    int32_t* tile_counts;  // [ceil(T/128)][2][N] per-tile histogram of the chosen experts by token parity, or null
     int T, fn, K, n_groups, topk_groups, group_topn, renorm, fused;
     int bias_in_logits;  // the bias joins the logit offset; the selection key is the score itself
     float scale;
@@ -187,6 +189,7 @@ struct Xch {
     float* ls;    // [BM][8]
     int* li;      // [BM][8]
     int* agree;   // [2][EPI_WARPS]: per tile parity, each warp's wait verdict
+    int* hist;    // [2][BN]: the tile's chosen experts counted by token parity (fused, tile_counts given)
 };
 
 // One token row (this thread's TMEM lane) of one finished tile.  The two
@@ -306,7 +309,29 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
     if (h == 0) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) top.offer(x.lk[row * 8 + j], x.li[row * 8 + j], x.ls[row * 8 + j]);
-        if (live) top.write(p.K, p.renorm, p.scale, p.idx + grow * p.K, p.w + grow * p.K);
+        if (live) {
+            top.write(p.K, p.renorm, p.scale, p.idx + grow * p.K, p.w + grow * p.K);
+            if (p.tile_counts != nullptr) {
+                int* hp = x.hist + (int)(grow & 1) * BN;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < p.K && (unsigned)top.i[k] < (unsigned)BN) atomicAdd(hp + top.i[k], 1);
+            }
+        }
+    }
+}
+
+// After a fused tile's rows: its histogram to global memory (tile index
+// `tile`, skipped past the last token), and cleared for the next tile.  Every
+// epilogue thread calls it; the named barrier orders the rows' counts first.
+template <int BN>
+__device__ __forceinline__ void flush_tile_hist(const Epi& p, const Xch& x, int64_t tile) {
+    epi_sync();
+    const int et = (int)threadIdx.x - 64;  // epilogue threads are warps 2..
+    int32_t* dst = tile * BM < (int64_t)p.T ? p.tile_counts + tile * 2 * BN : nullptr;
+    for (int i = et; i < 2 * BN; i += EPI_THREADS) {
+        if (dst != nullptr) dst[i] = x.hist[i];
+        x.hist[i] = 0;
     }
 }
 
@@ -332,12 +357,14 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     xch.ls = xch.lk + 8 * BM;
     xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
     xch.agree = xch.li + 8 * BM;
+    xch.hist = xch.agree + 2 * EPI_WARPS;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
     const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
     const int num_kb = (d + BK - 1) / BK;
+    for (int i = threadIdx.x; i < 2 * BN; i += blockDim.x) xch.hist[i] = 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
@@ -436,6 +463,7 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty0 + 8 * a);
+            if (FUSED && p.tile_counts != nullptr) flush_tile_hist<BN>(p, xch, tile);
         }
     }
 
@@ -550,6 +578,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     xch.ls = xch.lk + 8 * BM;
     xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
     xch.agree = xch.li + 8 * BM;
+    xch.hist = xch.agree + 2 * EPI_WARPS;
+    for (int i = threadIdx.x; i < 2 * BN; i += blockDim.x) xch.hist[i] = 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -658,6 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * a);
+            if (FUSED && p.tile_counts != nullptr) flush_tile_hist<BN>(p, xch, (int64_t)tp * 2 + rank);
         }
     }
 
@@ -760,8 +791,9 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
 cudaError_t launch_gate_tc(const void* x, const void* W, const float* off, const float* bias, int T, int d, int N,
                            int K, int fn, int n_groups, int topk_groups, int group_topn, int renorm, float scale,
                            bool fused, bool bias_in_logits, float* scores, int32_t* idx, float* w, int32_t* err,
-                           int max_ctas, cudaStream_t st) {
+                           int max_ctas, int32_t* tile_counts, cudaStream_t st) {
     tc::Epi p;
+    p.tile_counts = fused ? tile_counts : nullptr;
     p.bias_in_logits = bias_in_logits ? 1 : 0;
     p.off = off; p.bias = bias; p.scores = scores; p.idx = idx; p.w = w;
     p.T = T; p.fn = fn; p.K = K; p.n_groups = n_groups; p.topk_groups = topk_groups; p.group_topn = group_topn;

@@ -98,17 +98,22 @@ __device__ __forceinline__ int ld_volatile(const int32_t* p) { return *reinterpr
 // ---------------------------------------------------------------------------
 // counts, offsets and statistics from the totals (the last block's
 // inclusive prefix over blocks); one combined block reduction for the stats
-__device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, int64_t A, int32_t* __restrict__ counts,
-                                              int32_t* __restrict__ offsets, moe_stats* stats,
-                                              const double* __restrict__ hs_partial, int hs_blocks, int N, int64_t T,
-                                              const ScanCtl* ctl, int* s_scan, double* s_red, int* s_cnt) {
+// tot: the totals, in global memory (read through L2) or, when tot_shared,
+// in this block's shared memory; err_word (may be null) holds the call's
+// error bits, or'ed with local_err
+__device__ __forceinline__ void finish_totals(const int32_t* tot, bool tot_shared, int n_slots, int64_t A,
+                                              int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                              moe_stats* stats, const double* __restrict__ hs_partial, int hs_blocks,
+                                              int N, int64_t T, const int32_t* err_word, int local_err, int* s_scan,
+                                              double* s_red, int* s_cnt) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int c8[LS_SLOTS_PER_THREAD];
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
         const int e = tid * LS_SLOTS_PER_THREAD + j;
-        c8[j] = e < n_slots ? __ldcg(tot + e) : 0;
+        c8[j] = e < n_slots ? (tot_shared ? tot[e] : __ldcg(tot + e)) : 0;
     }
+    __syncthreads();  // every total read before s_cnt (which may alias tot) is written
     int tsum = 0;
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) tsum += c8[j];
@@ -169,7 +174,7 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, int n_slots, i
             rHs += s_red[24 + w];
         }
         rvar /= (double)(n_slots > 0 ? n_slots : 1);
-        const int err = ld_volatile(&ctl->err);
+        const int err = (err_word != nullptr ? ld_volatile(err_word) : 0) | local_err;
         stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
         stats->n_slots = n_slots;
         stats->total = (int64_t)total_i;
@@ -391,11 +396,238 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
     if (b == nblk - 1 && counts != nullptr) {  // (the bounded-wait self-test passes no outputs)
         __syncthreads();
         // the warp histograms are no longer needed: they hold the counts for the statistics
-        finish_totals(pre + b * n_slots, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T, ctl,
-                      s_scan, s_red, wh);
+        finish_totals(pre + b * n_slots, false, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T,
+                      &ctl->err, 0, s_scan, s_red, wh);
     }
     __syncthreads();
     block_done(ctl, nblk);
+}
+
+// ---------------------------------------------------------------------------
+// Load statistics without a look-back chain (problems up to ~2.6M
+// assignments).  Block b takes assignments [b*BPB, (b+1)*BPB), BPB = 8 warps x
+// C chunks of 32 (one wave of at most ~320 blocks):
+//  1. slots, warp histograms and in-warp stable ranks, as above;
+//  2. per-slot prefix over the block's warps; the block's per-slot counts are
+//     published as 64-bit words whose high half carries this call's tag
+//     (bit 31 | epoch), so a word is its own ready flag: no separate flag and
+//     no fence on the normal path (a word without the tag -- zero, an older
+//     call's, or another layout's int32 data, which never has bit 31 in that
+//     half -- reads as "not yet");
+//  3. each block sums, per slot, the words of ALL earlier blocks (independent
+//     loads, a bounded re-poll of any word not yet tagged): the count of every
+//     earlier assignment in that slot, without waiting on inclusive prefixes;
+//  4. rank = earlier blocks + earlier warps + within the warp;
+//  5. the last block's sums plus its own counts are the totals: counts,
+//     offsets, statistics.  The last block to finish advances the epoch.
+// A one-block problem shares nothing with other blocks: it publishes nothing,
+// waits for nothing and leaves the control words untouched (error bits go to
+// the sticky word directly).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+template <int C>
+__global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
+    const int32_t* __restrict__ idx, int64_t A, int K, int N, const int32_t* __restrict__ replica_slot,
+    int n_slots, int32_t* __restrict__ slot_out, int32_t* __restrict__ rank_out, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, moe_stats* stats, const double* __restrict__ hs_partial, int hs_blocks,
+    int64_t T, ScanCtl* ctl, uint64_t* agg64, int nblk, int block_base, const int32_t* __restrict__ tile_counts) {
+    constexpr int BPB = LS_WARPS * C * 32;
+    extern __shared__ int32_t sm_dyn[];
+    int32_t* wh = sm_dyn;                       // [LS_WARPS][n_slots]
+    int32_t* ex = sm_dyn + LS_WARPS * n_slots;  // [n_slots] earlier-block counts
+    __shared__ int s_err;
+    __shared__ int s_scan[33];
+    __shared__ double s_red[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = block_base + (int)blockIdx.x;  // block_base > 0 only in the bounded-wait self-test
+    const bool multi = nblk > 1;
+
+    // the loads first: expert ids of this warp's chunks, and the call's epoch
+    const int64_t base_a = (int64_t)b * BPB + (int64_t)warp * (C * 32);
+    int slot_r[C], rank_r[C];
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        slot_r[j] = a < A ? __ldg(idx + a) : -1;
+    }
+    const uint32_t tag = multi ? (0x80000000u | (uint32_t)ld_volatile(reinterpret_cast<const int32_t*>(&ctl->epoch)))
+                               : 0u;
+    if (tid == 0) s_err = 0;
+    for (int i = tid; i < LS_WARPS * n_slots; i += LS_THREADS) wh[i] = 0;
+    // the gate epilogue's per-tile histograms (tiles of 128 tokens, aligned to
+    // this block, split by token parity) give the block's counts without its
+    // indices: publish them at once
+    const bool pre_published = tile_counts != nullptr && multi;
+    int tc_agg[LS_SLOTS_PER_THREAD];
+    if (pre_published) {
+        const int64_t tok0 = (int64_t)b * (BPB / K);
+        const int64_t ntiles = (T + 127) / 128;
+        const int64_t j0 = tok0 / 128;
+        const int64_t j1 = min(ntiles, j0 + (int64_t)(BPB / K) / 128);
+        // replica slot -> the expert it copies (ex[] is free until step 3)
+        for (int i = tid; i < n_slots - N; i += LS_THREADS) ex[i] = -1;
+        __syncthreads();
+        if (replica_slot != nullptr)
+            for (int e = tid; e < N; e += LS_THREADS) {
+                const int r = __ldg(replica_slot + e);
+                if (r >= N && r < n_slots) ex[r - N] = e;
+            }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+            const int e = tid + j * LS_THREADS;
+            int c = 0;
+            if (e < n_slots) {
+                const int src = e < N ? e : ex[e - N];
+                const bool has_rep = e < N && replica_slot != nullptr && __ldg(replica_slot + e) >= 0;
+                if (src >= 0)
+                    for (int64_t q = j0; q < j1; ++q) {
+                        const int32_t* tq = tile_counts + q * 2 * N;
+                        if (e < N) c += __ldg(tq + src) + (has_rep ? 0 : __ldg(tq + N + src));
+                        else c += __ldg(tq + N + src);
+                    }
+                if (b < nblk - 1) st_relaxed_u64(agg64 + (int64_t)b * n_slots + e, ((uint64_t)tag << 32) | (uint32_t)c);
+            }
+            tc_agg[j] = c;
+        }
+    }
+    __syncthreads();
+
+    // 1. slots, warp histograms, in-warp stable ranks
+    int32_t* my = wh + warp * n_slots;
+    int bad = 0;
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        int slot = slot_r[j];
+        if (a < A) {
+            if (slot < 0) {
+                slot = -1;  // dropped by the capacity limit: no slot, rank -1
+            } else if (slot >= N) {
+                bad = 1;
+                slot = -1;
+            } else if (replica_slot != nullptr) {
+                const int r = __ldg(replica_slot + slot);
+                if (r >= 0 && ((a / K) & 1)) slot = r;
+                if (slot >= n_slots) { bad = 1; slot = -1; }
+            }
+            if (slot_out != nullptr) slot_out[a] = slot;
+        }
+        const unsigned peers = __match_any_sync(FULL, slot);
+        const int before = __popc(peers & lanemask_lt());
+        const int seen = (slot >= 0) ? my[slot] : 0;
+        __syncwarp();
+        if (slot >= 0 && before == 0) my[slot] = seen + __popc(peers);
+        __syncwarp();
+        slot_r[j] = slot;
+        rank_r[j] = seen + before;
+    }
+    if (__any_sync(FULL, bad) && lane == 0) atomicOr(&s_err, 2);
+    __syncthreads();
+    const int blk_err = s_err;
+    if (multi && blk_err != 0 && tid == 0) {
+        // rare path: the error bit is visible before this block's counts are
+        atomicOr(&ctl->err, blk_err);
+        __threadfence();
+    }
+    __syncthreads();
+
+    // 2. per-slot exclusive prefix over warps; the block's counts, published
+    int my_agg[LS_SLOTS_PER_THREAD];
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid + j * LS_THREADS;
+        my_agg[j] = 0;
+        if (e < n_slots) {
+            int run = 0;
+#pragma unroll
+            for (int w = 0; w < LS_WARPS; ++w) {
+                const int c = wh[w * n_slots + e];
+                wh[w * n_slots + e] = run;
+                run += c;
+            }
+            my_agg[j] = run;
+            if (pre_published) {
+                if (tc_agg[j] != run) atomicOr(&s_err, 2);  // the tile histograms do not match the indices
+            } else if (multi && b < nblk - 1) {
+                st_relaxed_u64(agg64 + (int64_t)b * n_slots + e, ((uint64_t)tag << 32) | (uint32_t)run);
+            }
+        }
+    }
+
+    // 3. counts of all earlier blocks, per slot: 8 independent loads at a time
+    int excl[LS_SLOTS_PER_THREAD];
+    bool timed_out = false;
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        excl[j] = 0;
+        const int e = tid + j * LS_THREADS;
+        if (e >= n_slots || b == 0) continue;
+        uint64_t t0 = 0;
+        for (int q0 = 0; q0 < b; q0 += 8) {
+            uint64_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = q0 + u < b ? ld_relaxed_u64(agg64 + (int64_t)(q0 + u) * n_slots + e) : ((uint64_t)tag << 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                // bounded re-poll of a word this call's block q0+u has not published yet
+                while ((uint32_t)(v[u] >> 32) != tag && !timed_out) {
+                    if (t0 == 0) t0 = globaltimer();
+                    else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
+                    __nanosleep(64);
+                    v[u] = ld_relaxed_u64(agg64 + (int64_t)(q0 + u) * n_slots + e);
+                }
+                excl[j] += (uint32_t)(v[u] >> 32) == tag ? (int)(uint32_t)v[u] : 0;
+            }
+        }
+    }
+    if (timed_out) atomicOr(&s_err, 1);
+#pragma unroll
+    for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+        const int e = tid + j * LS_THREADS;
+        if (e < n_slots) ex[e] = excl[j];
+    }
+    __syncthreads();
+
+    // 4. in-expert ranks
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+        const int64_t a = base_a + j * 32 + lane;
+        if (a < A) rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+    }
+
+    // 5. the last block: totals = earlier blocks + its own counts
+    if (b == nblk - 1 && counts != nullptr) {
+        const int local_err = s_err;
+        if (multi) __threadfence();  // other blocks' error bits, published before their counts, are visible
+        __syncthreads();             // ranks read ex and my before wh is reused for the totals
+#pragma unroll
+        for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
+            const int e = tid + j * LS_THREADS;
+            if (e < n_slots) wh[e] = excl[j] + my_agg[j];
+        }
+        __syncthreads();
+        finish_totals(wh, true, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T,
+                      multi ? &ctl->err : nullptr, local_err, s_scan, s_red, wh);
+    }
+    if (multi) {
+        __syncthreads();
+        if (tid == 0 && (s_err & ~blk_err)) atomicOr(&ctl->err, s_err & ~blk_err);  // timeouts, histogram mismatch
+        __syncthreads();
+        block_done(ctl, nblk);
+    } else if (tid == 0 && s_err != 0) {
+        atomicOr(&ctl->sticky, s_err);  // read and cleared by moe_workspace_status
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -506,7 +738,7 @@ __global__ void __launch_bounds__(256) route_balanced_kernel(int64_t A, int K, i
 cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const int32_t* replica_slot,
                               int n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets,
                               int32_t* rank, const float* scores, int score_fn, moe_stats* stats,
-                              void* ws, cudaStream_t st) {
+                              void* ws, cudaStream_t st, const int32_t* tile_counts) {
     const WsLayout L = ws_layout(T, K, N, n_slots);
     char* w = static_cast<char*>(ws);
     ScanCtl* ctl = reinterpret_cast<ScanCtl*>(w + L.ctl);
@@ -529,6 +761,27 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
         part = partial;
     }
     const size_t lsm = sizeof(int32_t) * (LS_WARPS + 1) * (size_t)n_slots;
+    // problems of up to V2_MAX_BLOCKS blocks of 2048, 4096 or 8192 assignments
+    // run without a look-back chain; larger ones use the look-back kernel
+    const int chunks = A <= (int64_t)V2_MAX_BLOCKS / 2 * 2048 ? 8 : (A <= (int64_t)V2_MAX_BLOCKS / 2 * 4096 ? 16 : 32);
+    const int64_t nb2 = (A + (int64_t)LS_THREADS * chunks - 1) / ((int64_t)LS_THREADS * chunks);
+    if (nb2 <= V2_MAX_BLOCKS) {
+        const int nb = nb2 < 1 ? 1 : (int)nb2;
+        uint64_t* agg64 = reinterpret_cast<uint64_t*>(agg);  // the agg and pre regions hold 8 bytes per cell
+        auto kern = chunks == 8 ? load_stats_v2_kernel<8> : (chunks == 16 ? load_stats_v2_kernel<16>
+                                                                          : load_stats_v2_kernel<32>);
+        if (lsm > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm);
+            if (e != cudaSuccess) return e;
+        }
+        // the tile histograms serve when a block is a whole number of 128-token tiles
+        const int bpb = LS_THREADS * chunks;
+        const bool tiles_ok = tile_counts != nullptr && bpb % K == 0 && (bpb / K) % 128 == 0;
+        kern<<<nb, LS_THREADS, lsm, st>>>(idx, A, K, N, replica_slot, n_slots, slot_idx, rank, counts, offsets, stats,
+                                          part, HS_BLOCKS, T, ctl, agg64, nb, 0, tiles_ok ? tile_counts : nullptr);
+        moe_host::note_launch();
+        return cudaGetLastError();
+    }
     if (lsm > 48 * 1024) {
         e = cudaFuncSetAttribute(load_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm);
         if (e != cudaSuccess) return e;
@@ -540,35 +793,50 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
     return cudaGetLastError();
 }
 
-// Self-test of the bounded look-back wait: a two-block problem (no
-// assignments, 8 slots) of which only the second block is launched, so the
-// flag of block 0 is never set.  The block must give up after the wait limit,
-// set the timeout bit and finish.  Returns the error bits read back.
+// Self-test of the bounded waits of both load-statistics kernels: a
+// two-block problem (no assignments, 8 slots) of which only the second block
+// is launched, so block 0 never publishes (its look-back flag, or its tagged
+// counts, never appear).  Each probe block must give up after the wait
+// limit, set the timeout bit and finish.  Returns the error bits of the two
+// probes and'ed (bit 0 set only if both waits ran out).
 cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t st) {
     const WsLayout L = ws_layout(2 * LS_BLOCK, 1, 8, 8);
     char* w = static_cast<char*>(ws);
     ScanCtl* ctl = reinterpret_cast<ScanCtl*>(w + L.ctl);
-    // ticket, finished count and error words start at zero; the epoch stays,
-    // so flags left by earlier calls are stale for the probe
-    cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
-    if (e != cudaSuccess) return e;
-    load_stats_kernel<<<1, LS_THREADS, sizeof(int32_t) * (LS_WARPS + 1) * 8, st>>>(
-        nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,
-        reinterpret_cast<uint32_t*>(w + L.flags), reinterpret_cast<int32_t*>(w + L.agg),
-        reinterpret_cast<int32_t*>(w + L.pre), /*nblk=*/2, /*ticket_base=*/1u);
-    moe_host::note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ScanCtl h;
-    if ((e = cudaMemcpyAsync(&h, ctl, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return e;
-    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
-    *err_out = h.err | h.sticky;  // the probe's block is also the last to finish: it folds err into sticky
-    // leave the workspace as a finished call does: counters zero, next epoch
-    // (the probe's own flag becomes stale), error words cleared
-    ScanCtl z;
-    memset(&z, 0, sizeof(z));
-    z.epoch = h.epoch + 1;
-    if ((e = cudaMemcpyAsync(ctl, &z, sizeof(z), cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
-    return cudaStreamSynchronize(st);
+    int32_t bits = ~0;
+    for (int probe = 0; probe < 2; ++probe) {
+        // ticket, finished count and error words start at zero; the epoch
+        // stays, so flags and tagged counts left by earlier calls are stale
+        cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
+        if (e != cudaSuccess) return e;
+        const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8;
+        if (probe == 0)
+            load_stats_kernel<<<1, LS_THREADS, smem, st>>>(
+                nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,
+                reinterpret_cast<uint32_t*>(w + L.flags), reinterpret_cast<int32_t*>(w + L.agg),
+                reinterpret_cast<int32_t*>(w + L.pre), /*nblk=*/2, /*ticket_base=*/1u);
+        else
+            load_stats_v2_kernel<8><<<1, LS_THREADS, smem, st>>>(
+                nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,
+                reinterpret_cast<uint64_t*>(w + L.agg), /*nblk=*/2, /*block_base=*/1, nullptr);
+        moe_host::note_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        ScanCtl h;
+        if ((e = cudaMemcpyAsync(&h, ctl, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return e;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+        // the look-back probe's block is also the last to finish (it folds err
+        // into sticky); the other probe's finished count stops short of 2
+        bits &= h.err | h.sticky;
+        // leave the workspace as a finished call does: counters zero, next
+        // epoch (the probe's own flags become stale), error words cleared
+        ScanCtl z;
+        memset(&z, 0, sizeof(z));
+        z.epoch = h.epoch + 1;
+        if ((e = cudaMemcpyAsync(ctl, &z, sizeof(z), cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
+        if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+    }
+    *err_out = bits;
+    return cudaSuccess;
 }
 
 cudaError_t launch_replica_plan(const int32_t* counts, int N, int R, int32_t* replica_slot, cudaStream_t st) {

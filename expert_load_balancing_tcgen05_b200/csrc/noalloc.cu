@@ -18,8 +18,8 @@
 // leaves its control words (tile ticket, finished-block count, error words,
 // call epoch) reset when its last block finishes, but a call must not depend
 // on the previous one having ended cleanly, so every call here first clears,
-// on its own stream, the control block and the look-back flags of its
-// layout (a few KB).  Two calls whose kernels overlap on the GPU race on the
+// on its own stream, the control block, look-back flags and per-block count
+// words of its layout (at most about 1.2 MB).  Two calls whose kernels overlap on the GPU race on the
 // array; the caller must serialise them.
 #include <mutex>
 
@@ -28,7 +28,8 @@
 namespace moe {
 cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const int32_t* replica_slot,
                               int n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets, int32_t* rank,
-                              const float* scores, int score_fn, moe_stats* stats, void* ws, cudaStream_t st);
+                              const float* scores, int score_fn, moe_stats* stats, void* ws, cudaStream_t st,
+                              const int32_t* tile_counts = nullptr);
 }
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
@@ -72,10 +73,12 @@ extern "C" moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T,
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // control block and look-back flags start at zero (the epoch restarts at
-    // 0, and the zeroed flags carry no tag of it)
+    // the control block, the look-back flags and the per-block count words
+    // start at zero: the epoch restarts at 0 and no word carries its tag
+    // (at most 1.2 MB for the largest workload here)
     const moe::WsLayout L = moe::ws_layout(T, K, N, n_slots);
-    if (cudaMemsetAsync(static_cast<char*>(ws) + L.ctl, 0, L.ctl_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(static_cast<char*>(ws) + L.ctl, 0, L.hs_partial - L.ctl, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
     const cudaError_t e = moe::launch_load_stats(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, counts, offsets,
                                                  rank, scores, score_fn, stats, ws, st);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

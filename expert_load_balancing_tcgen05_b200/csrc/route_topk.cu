@@ -12,6 +12,7 @@
 // every reduction is a butterfly of shuffles; nothing goes through shared
 // memory.  The order (key desc, index asc) is total, so the result is unique.
 #include <math.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "select.cuh"
@@ -422,6 +423,169 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-per-token selection.  Lane l owns experts [l*EPL, l*EPL + EPL)
+// (EPL = N/32), so an expert group of 32 spans G = 32/EPL consecutive lanes;
+// the lane's bias values live in registers for the whole kernel.
+//   1. keys = fp32(s + b); each lane's two largest keys (t1 >= t2);
+//   2. with groups: the group's two largest keys by a butterfly over its G
+//      lanes, group score fp32(t1 + t2) (or t1), group ranks from the
+//      scores of all groups (shuffles); lanes of groups not kept drop out;
+//   3. theta = the ceil(K/2)-th largest t2 over the kept lanes (ceil(K/2)
+//      rounds of a warp max-reduction, redux.sync, on order-preserving
+//      integer images of the keys).  At least ceil(K/2) kept lanes hold two
+//      keys >= theta, so at least K kept keys are >= theta and the K best
+//      keys are all >= theta;
+//   4. the survivors (kept keys >= theta; typically K to K+4) are written to
+//      a per-warp shared list in expert order, one per lane, and each lane
+//      ranks its survivor against the others (rank = how many beat it by key
+//      desc, list position asc = index asc); survivors of rank < K are
+//      placed at their rank; lanes 0..K-1 write the outputs, the weights
+//      from the unbiased scores summed in k order.  A token with more than
+//      32 survivors takes K rounds of a warp argmax instead.
+// The result is the plain definition's: the survivors contain the K best
+// kept keys and the ranking is the (key desc, index asc) order.
+// ---------------------------------------------------------------------------
+constexpr int SW_THREADS = 256;
+
+// order-preserving image of a float key in the unsigned integers (-0 and +0,
+// equal as keys, share one image)
+__device__ __forceinline__ uint32_t ord_key(float f) {
+    const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(SW_THREADS) route_select_warp_kernel(
+    const float* __restrict__ scores, const float* __restrict__ bias, int T, int K, int grouped, int topk_groups,
+    int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    constexpr int N = 32 * EPL;
+    constexpr int G = 32 / EPL;  // lanes per group of 32 experts
+    __shared__ float l_key[SW_THREADS / 32][32], l_s[SW_THREADS / 32][32];
+    __shared__ int l_idx[SW_THREADS / 32][32];
+    __shared__ float o_s[SW_THREADS / 32][8];
+    __shared__ int o_i[SW_THREADS / 32][8];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int e0 = lane * EPL;
+    float b[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) b[i] = bias != nullptr ? __ldg(bias + e0 + i) : 0.f;
+    const int rounds = (K + 1) >> 1;
+    const int warps = gridDim.x * (SW_THREADS / 32);
+
+    for (int64_t t = (int64_t)blockIdx.x * (SW_THREADS / 32) + wib; t < T; t += warps) {
+        float sv[EPL], kv[EPL];
+        load_row<EPL>(scores + t * N, lane, N, sv);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) kv[i] = __fadd_rn(sv[i], b[i]);
+        // 1. the lane's two largest keys
+        float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            t2 = kv[i] > t1 ? t1 : (kv[i] > t2 ? kv[i] : t2);
+            t1 = kv[i] > t1 ? kv[i] : t1;
+        }
+        // 2. groups: the group's top two over its lanes, scores, ranks
+        bool kept = true;
+        if (grouped) {
+            float g1 = t1, g2 = t2;
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1) {
+                const float h1 = __shfl_xor_sync(FULL, g1, o), h2 = __shfl_xor_sync(FULL, g2, o);
+                const float lo = fminf(g1, h1);
+                g1 = fmaxf(g1, h1);
+                g2 = fmaxf(lo, fmaxf(g2, h2));
+            }
+            const float gs = group_topn == 1 ? g1 : __fadd_rn(g1, g2);
+            const int g = lane / G;
+            int rank = 0;
+#pragma unroll
+            for (int h = 0; h < EPL; ++h) {  // EPL = number of groups of 32
+                const float gh = __shfl_sync(FULL, gs, h * G);
+                rank += (h != g && beats(gh, h, gs, g)) ? 1 : 0;
+            }
+            kept = rank < topk_groups;
+        }
+        // 3. theta: the ceil(K/2)-th largest t2 over the kept lanes
+        uint32_t u2 = kept ? ord_key(t2) : 0u, th_u = 0u;
+        for (int r = 0; r < rounds; ++r) {
+            th_u = __reduce_max_sync(FULL, u2);
+            if (u2 == th_u) u2 = 0u;
+        }
+        // 4. survivors, compacted in expert order
+        unsigned m = 0;
+        if (kept) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) m |= (ord_key(kv[i]) >= th_u ? 1u : 0u) << i;
+        }
+        const int cnt = __popc(m);
+        const int total = __reduce_add_sync(FULL, (unsigned)cnt);
+        if (total <= 32) {
+            int off = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(FULL, off, o);
+                if (lane >= o) off += y;
+            }
+            off -= cnt;
+            while (m) {
+                const int i = __ffs(m) - 1;
+                m &= m - 1;
+#pragma unroll
+                for (int q = 0; q < EPL; ++q)
+                    if (q == i) {
+                        l_key[wib][off] = kv[q];
+                        l_s[wib][off] = sv[q];
+                    }
+                l_idx[wib][off] = e0 + i;
+                ++off;
+            }
+            __syncwarp();
+            const float kc = lane < total ? l_key[wib][lane] : -INFINITY;
+            int rank = 0;
+            for (int c2 = 0; c2 < total; ++c2) {
+                const float k2 = l_key[wib][c2];
+                rank += (k2 > kc || (k2 == kc && c2 < lane)) ? 1 : 0;
+            }
+            if (lane < total && rank < K) {
+                o_i[wib][rank] = l_idx[wib][lane];
+                o_s[wib][rank] = l_s[wib][lane];
+            }
+            __syncwarp();
+        } else {
+            // more survivors than lanes: K rounds of a warp argmax over them
+            int my_i = 0;
+            float my_s = 0.f;
+            for (int k = 0; k < K; ++k) {
+                float bk = -INFINITY, bs = 0.f;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (((m >> i) & 1u) && beats(kv[i], e0 + i, bk, bi)) { bk = kv[i]; bi = e0 + i; bs = sv[i]; }
+                float wk = bk;
+                int wi = bi;
+                argmax_span(wk, wi, 32);
+                const int owner = wi / EPL;
+                const float ws = __shfl_sync(FULL, bs, owner);
+                if (lane == owner) m &= ~(1u << (wi - e0));
+                if (lane == k) { my_i = wi; my_s = ws; }
+            }
+            if (lane < K) { o_i[wib][lane] = my_i; o_s[wib][lane] = my_s; }
+            __syncwarp();
+        }
+        // outputs: weights from the unbiased scores, summed in k order
+        if (lane < K) {
+            float ssum = o_s[wib][0];
+            for (int k = 1; k < K; ++k) ssum = __fadd_rn(ssum, o_s[wib][k]);
+            const float sk = o_s[wib][lane];
+            const float wv = renorm ? __fdiv_rn(sk, ssum) : sk;
+            topk_idx[t * K + lane] = o_i[wib][lane];
+            topk_w[t * K + lane] = __fmul_rn(wv, route_scale);
+        }
+        __syncwarp();
+    }
+}
+
 // The filtered kernel covers N in {64, 128, 256}, K <= 8, and either one
 // group or groups of exactly 32 experts with a group score of the top one or
 // two keys, when the candidate threads hold at least K known keys (2 each).
@@ -442,9 +606,38 @@ int route_epl(int N) {
     return 0;
 }
 
+// The warp-per-token kernel covers N in {64, 128, 256, 512}, K <= 8, and
+// either one group or groups of exactly 32 experts with a group score of the
+// top one or two keys.
+static bool select_warp_ok(int N, int K, int n_groups, int group_topn) {
+    if (!(N == 64 || N == 128 || N == 256 || N == 512) || K > 8) return false;
+    return n_groups == 1 || (N / n_groups == 32 && group_topn >= 1 && group_topn <= 2);
+}
+
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K,
                               int n_groups, int topk_groups, int group_topn, int renorm,
                               float route_scale, int32_t* idx, float* w, cudaStream_t st) {
+    const char* env = getenv("MOE_SELECT_KERNEL");  // "filtered": the thread-per-group kernel (measurement)
+    const bool filtered = env != nullptr && env[0] == 'f';
+    if (!filtered && select_warp_ok(N, K, n_groups, group_topn)) {
+        long long blocks = ((long long)T + SW_THREADS / 32 - 1) / (SW_THREADS / 32);
+        const long long cap = (long long)moe_host::sm_count() * 8;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+        const int grouped = n_groups > 1 ? 1 : 0;
+#define MOE_SELW(E)                                                                                            \
+    route_select_warp_kernel<E><<<(unsigned)blocks, SW_THREADS, 0, st>>>(scores, bias, T, K, grouped, topk_groups, \
+                                                                         group_topn, renorm, route_scale, idx, w)
+        switch (N) {
+            case 64: MOE_SELW(2); break;
+            case 128: MOE_SELW(4); break;
+            case 256: MOE_SELW(8); break;
+            default: MOE_SELW(16); break;
+        }
+#undef MOE_SELW
+        moe_host::note_launch();
+        return cudaGetLastError();
+    }
     if (select_fast_ok(N, K, n_groups, topk_groups, group_topn)) {
         const int S = N / 32;
         long long blocks = ((long long)T * S + SEL_THREADS - 1) / SEL_THREADS;

@@ -29,7 +29,8 @@ MOE_F32, MOE_BF16 = 0, 1
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_load_stats", "moe_replica_plan", "moe_bias_update",
            "moe_dispatch", "moe_combine", "moe_workspace_status", "moe_launch_count", "moe_status_str",
            "moe_version", "moe_load_stats_noalloc", "moe_selftest_wait_timeout", "moe_route_balanced",
-           "moe_bias_update_ema", "moe_route_capacity", "moe_capacity_workspace_bytes", "moe_capacity_limit")
+           "moe_bias_update_ema", "moe_route_capacity", "moe_capacity_workspace_bytes", "moe_capacity_limit",
+           "moe_route_tiles", "moe_load_stats_tiles")
 
 
 class RouteCfg(ctypes.Structure):
@@ -129,6 +130,30 @@ def moe_load_stats_noalloc(topk_idx, T, K, N, replica_slot, n_slots, slot_idx, c
     _check(_lib.moe_load_stats_noalloc(_ptr(topk_idx), T, K, N, _ptr(replica_slot), n_slots, _ptr(slot_idx),
                                        _ptr(counts), _ptr(offsets), _ptr(rank), _ptr(scores), score_fn,
                                        _ptr(stats), _stream(stream)), "moe_load_stats_noalloc")
+
+
+_lib.moe_route_tiles.argtypes = [ctypes.POINTER(RouteCfg), _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_route_tiles.restype = _I32
+_lib.moe_load_stats_tiles.argtypes = [_P, _I64, _I32, _I32, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_load_stats_tiles.restype = _I32
+
+
+def tile_counts_shape(T, N):
+    """Shape of the per-tile histograms of moe_route_tiles: [ceil(T/128), 2, N]."""
+    return ((T + 127) // 128, 2, N)
+
+
+def moe_route_tiles(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, tile_counts, ws, stream=None):
+    _check(_lib.moe_route_tiles(ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(bias),
+                                _ptr(topk_idx), _ptr(topk_w), _ptr(tile_counts), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "moe_route_tiles")
+
+
+def moe_load_stats_tiles(topk_idx, T, K, N, tile_counts, replica_slot, n_slots, slot_idx, counts, offsets, rank,
+                         stats, ws, stream=None):
+    _check(_lib.moe_load_stats_tiles(_ptr(topk_idx), T, K, N, _ptr(tile_counts), _ptr(replica_slot), n_slots,
+                                     _ptr(slot_idx), _ptr(counts), _ptr(offsets), _ptr(rank), _ptr(stats), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "moe_load_stats_tiles")
 
 
 _lib.moe_route_balanced.argtypes = [_I64, _I32, _I32, _F32, _P, _P, _P]

@@ -6,14 +6,18 @@ Two schedules of the same library calls:
 * serial -- the calls in order on the caller's stream;
 * pipelined -- the routing of batch i+1 (gate, selection, load statistics,
   bias step and, with several ranks, the all-reduce of the expert counts)
-  runs on a high-priority stream beside the dispatch of batch i on the
-  caller's stream.  Batch i+1 depends on batch i only through the bias,
-  which its routing stream updates in order, so every result equals the
-  serial schedule's.  The load-statistics outputs that dispatch reads
-  (slots, counts, offsets, ranks, stats) are double-buffered; a buffer set is
-  reused only after the dispatch that read it has finished.  The gate GEMM
+  runs on a high-priority stream beside the dispatch (and, when asked, the
+  combine) of batch i on the caller's stream.  Batch i+1 depends on batch i
+  only through the bias, which its routing stream updates in order, so every
+  result equals the serial schedule's.  Everything a batch's routing writes
+  and its dispatch or combine reads (scores, indices, weights, slots, counts,
+  offsets, ranks, stats) is double-buffered; a buffer set is reused only
+  after the dispatch and combine that read it have finished.  The gate GEMM
   gets a budget of SMs (``gate_max_ctas``) so that the dispatch, which is
   bound by HBM bandwidth, keeps the rest of the GPU.
+
+Combine runs on identity experts here (it gathers the dispatched rows back),
+the step having no expert FFNs.
 
 Host-side orchestration only: streams, events and buffers.  Every step of the
 path runs in the library's kernels.
@@ -35,17 +39,22 @@ class RoutingStep:
     different buffers, as in a stream of distinct batches)."""
 
     def __init__(self, wl, x, w_gate, bias, logit_offset, device, world: int = 1, pipelined: bool = True,
-                 gate_max_ctas: int | None = None, bias_rate: float = 0.001):
+                 gate_max_ctas: int | None = None, bias_rate: float = 0.001, fused: bool = False):
         T, d, N, K = wl.T, wl.d, wl.N, wl.K
         self.wl, self.dev, self.world, self.pipelined, self.u = wl, device, world, pipelined, bias_rate
+        # fused: the selection and a per-tile histogram in the gate's epilogue
+        # (moe_route_tiles, no scores in memory), statistics from those
+        # histograms (moe_load_stats_tiles)
+        self.fused = fused
         self.batches = list(x) if isinstance(x, (list, tuple)) else [x]
         x = self.batches[0]
         self.x, self.W, self.bias, self.off = x, w_gate, bias, logit_offset
         f32, i32 = torch.float32, torch.int32
-        self.scores = torch.empty(T, N, dtype=f32, device=device)
-        self.idx = torch.empty(T, K, dtype=i32, device=device)
-        self.w = torch.empty(T, K, dtype=f32, device=device)
-        self.sets = [dict(slot=torch.empty(T, K, dtype=i32, device=device),
+        self.sets = [dict(scores=(torch.empty(moe.tile_counts_shape(T, N), dtype=i32, device=device) if fused
+                                  else torch.empty(T, N, dtype=f32, device=device)),
+                          idx=torch.empty(T, K, dtype=i32, device=device),
+                          w=torch.empty(T, K, dtype=f32, device=device),
+                          slot=torch.empty(T, K, dtype=i32, device=device),
                           counts=torch.empty(N, dtype=i32, device=device),
                           offsets=torch.empty(N + 1, dtype=i32, device=device),
                           rank=torch.empty(T, K, dtype=i32, device=device),
@@ -72,12 +81,21 @@ class RoutingStep:
         wl = self.wl
         if stage_events is not None:
             stage_events[0].record(stream)
-        moe.moe_route(self.cfg, x, self.W, self.off, self.bias, self.scores, self.idx, self.w, self.ws,
-                      stream=stream)
+        if self.fused:
+            # s["scores"] holds the per-tile histograms on this path
+            moe.moe_route_tiles(self.cfg, x, self.W, self.off, self.bias, s["idx"], s["w"], s["scores"], self.ws,
+                                stream=stream)
+        else:
+            moe.moe_route(self.cfg, x, self.W, self.off, self.bias, s["scores"], s["idx"], s["w"], self.ws,
+                          stream=stream)
         if stage_events is not None:
             stage_events[1].record(stream)
-        moe.moe_load_stats(self.idx, wl.T, wl.K, wl.N, None, wl.N, s["slot"], s["counts"], s["offsets"], s["rank"],
-                           None, wl.fn, s["stats"], self.ws, stream=stream)
+        if self.fused:
+            moe.moe_load_stats_tiles(s["idx"], wl.T, wl.K, wl.N, s["scores"], None, wl.N, s["slot"], s["counts"],
+                                     s["offsets"], s["rank"], s["stats"], self.ws, stream=stream)
+        else:
+            moe.moe_load_stats(s["idx"], wl.T, wl.K, wl.N, None, wl.N, s["slot"], s["counts"], s["offsets"],
+                               s["rank"], None, wl.fn, s["stats"], self.ws, stream=stream)
         total = wl.T * wl.K
         if self.world > 1:
             # the bias is shared by every rank: its step uses the global counts
@@ -86,10 +104,26 @@ class RoutingStep:
             total *= self.world
         moe.moe_bias_update(s["counts"], wl.N, total, self.u, 0, self.bias, stream=stream)
 
-    def _dispatch_part(self, s, x, stream):
+    def _dispatch_part(self, s, x, stream, combine_out=None):
         wl = self.wl
         moe.moe_dispatch(x, wl.T, wl.d, wl.K, s["slot"], s["offsets"], s["rank"], self.rows, None, None, self.pos,
                          None, stream=stream)
+        if combine_out is not None:
+            # identity experts: the expert outputs are the dispatched rows
+            moe.moe_combine(self.rows, wl.T, wl.d, wl.K, self.pos, s["w"], combine_out, stream=stream)
+
+    # the last batch's routing outputs (scores: the per-tile histograms on the fused path)
+    @property
+    def scores(self):
+        return self.last()["scores"]
+
+    @property
+    def idx(self):
+        return self.last()["idx"]
+
+    @property
+    def w(self):
+        return self.last()["w"]
 
     # ------------------------------------------------------------------ api
     def fence(self):
@@ -100,14 +134,14 @@ class RoutingStep:
 
     def results(self, s):
         """The routing result of a batch: indices, weights, offsets, counts, stats."""
-        return [self.idx, self.w, s["offsets"], s["counts"], s["stats"]]
+        return [s["idx"], s["w"], s["offsets"], s["counts"], s["stats"]]
 
     def _copy_out(self, s, host_out, stream):
         with torch.cuda.stream(stream):
             for src, dst in zip(self.results(s), host_out):
                 dst.copy_(src, non_blocking=True)
 
-    def step(self, x=None, dispatch_events=None, stage_events=None, ready=None, host_out=None):
+    def step(self, x=None, dispatch_events=None, stage_events=None, ready=None, host_out=None, combine_out=None):
         """Enqueue one batch.
 
         x: the batch's tokens (default: the next of the batches given at
@@ -116,6 +150,9 @@ class RoutingStep:
         the host on another stream); host_out: pinned host tensors shaped like
         results(), filled with this batch's routing result (indices and
         weights are copied before the next batch overwrites them).
+        combine_out: optional [T, d] tensor; when given, the batch's rows are
+        combined back into it (identity experts) on the caller's stream
+        right after its dispatch.
         dispatch_events: optional (start, end) CUDA events recorded around the
         dispatch on the caller's stream.  stage_events (serial schedule only):
         four events recorded before the gate, after the selection, after the
@@ -133,7 +170,7 @@ class RoutingStep:
                 self._copy_out(s, host_out, main)
             if dispatch_events is not None:
                 dispatch_events[0].record(main)
-            self._dispatch_part(s, x, main)
+            self._dispatch_part(s, x, main, combine_out)
             if dispatch_events is not None:
                 dispatch_events[1].record(main)
             if stage_events is not None:
@@ -154,10 +191,10 @@ class RoutingStep:
         main.wait_event(self.ev_routed[b])
         if dispatch_events is not None:
             dispatch_events[0].record(main)
-        self._dispatch_part(s, x, main)
+        self._dispatch_part(s, x, main, combine_out)
         if dispatch_events is not None:
             dispatch_events[1].record(main)
-        self.ev_dispatched[b].record(main)
+        self.ev_dispatched[b].record(main)  # buffer set b: its dispatch and combine are done with it
         self.i += 1
 
     def last(self):

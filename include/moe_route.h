@@ -135,7 +135,13 @@ size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
  *   topk_groups groups with the best fp32 sum of their group_topn largest
  *   keys are kept and the rest excluded; the K best keys among the kept
  *   experts are chosen.  Order: key descending, ties to the lower index.
- *   topk_idx [T,K] int32 in that order.
+ *   topk_idx [T,K] int32 in that order.  Keys must be finite (scores and
+ *   bias finite, hence no NaN or infinite key): the pages define no order
+ *   for NaN, and with a non-finite key the choice is unspecified -- an
+ *   entry may even hold an id outside [0, N), which the load statistics
+ *   reject (an id >= N: stats->status = MOE_ERR_INVALID; a negative id
+ *   counts as dropped; either way slot -1 and nothing dispatched for it).
+ *   No path reads or writes out of bounds.
  * Weights ([ENT] "Concrete Implementation" renormalisation; [HD] weighted
  * combine by affinity): from the UNBIASED scores,
  *   topk_w[t,k] = fp32(fp32(s_k / fp32-sum-in-k-order) * route_scale)
@@ -146,6 +152,27 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
                      const float* logit_offset, const float* bias, float* scores,
                      int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
                      moe_stream_t stream);
+
+/*
+ * moe_route_tiles -- moe_route with the selection in the GEMM epilogue and
+ * the load histogram counted there too, per tile ([GL] section 6: fuse the
+ * routing computation with the dispatch path; the scores never reach
+ * memory).
+ * Same routing as moe_route (the tensor-core gate with the epilogue
+ * selection: bf16, N in {64, 128, 256}, K <= 8, one group or sigmoid groups
+ * of 32 experts with group_topn <= 2; otherwise MOE_ERR_UNSUPPORTED).  No
+ * scores are written.  Additionally, for every tile of 128 tokens,
+ *   tile_counts[j][p][e] = #{(t,k) : t in [128j, 128j+128), t % 2 == p,
+ *                           topk_idx[t,k] == e}
+ * (tile_counts int32 [ceil(T/128)][2][N]): the tile's expert histogram split
+ * by token parity, so that per-slot counts with replicas (odd tokens of a
+ * replicated expert go to its replica) follow without the indices.
+ * moe_load_stats_tiles takes them.
+ */
+moe_status moe_route_tiles(const moe_route_cfg* cfg, const void* x, const void* w_gate,
+                           const float* logit_offset, const float* bias, int32_t* topk_idx,
+                           float* topk_w, int32_t* tile_counts, void* ws, size_t ws_bytes,
+                           moe_stream_t stream);
 
 /*
  * moe_route_balanced -- "forcible load balancing": the top-K output replaced
@@ -222,10 +249,13 @@ moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, con
  * stats (device, may be NULL): see moe_stats.  scores [T,N] fp32 (may be
  *   NULL) adds entropy_score_bits, with score_fn telling softmax rows
  *   (used as they are) from sigmoid rows (normalised per token).
- * One single-pass kernel: blocks of 2048 assignments publish their per-slot
- * counts and look back over earlier blocks' count vectors (decoupled
- * look-back) for the ranks; the last block to finish writes counts, offsets
- * and stats.  Its waits are bounded (stats->status = MOE_ERR_TIMEOUT on
+ * One single-pass kernel.  Up to about 2.6M assignments (T*K): one wave of
+ * blocks of 2048, 4096 or 8192 assignments; each block publishes its
+ * per-slot counts as words tagged with the call, and sums the tagged counts
+ * of all earlier blocks for its ranks (no chain of prefixes); the last block
+ * writes counts, offsets and stats.  Larger problems: blocks of 2048
+ * assignments with a decoupled look-back over earlier blocks' count vectors.
+ * Either way the waits are bounded (stats->status = MOE_ERR_TIMEOUT on
  * expiry).
  */
 moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
@@ -233,6 +263,24 @@ moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t
                           int32_t* counts, int32_t* offsets, int32_t* rank,
                           const float* scores, int32_t score_fn, moe_stats* stats, void* ws,
                           size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_load_stats_tiles -- moe_load_stats (without the score entropy) for a
+ * routing made by moe_route_tiles, taking its per-tile histograms
+ * tile_counts [ceil(T/128)][2][N] as well as topk_idx.  Results are those of
+ * moe_load_stats.  Where a block of the statistics kernel is a whole number
+ * of 128-token tiles (K dividing 16, and up to about 2.6M assignments) the
+ * block's per-slot counts come from the tile histograms, so it publishes them
+ * to the later blocks before reading a single index; its own count of the
+ * indices is then checked against them (a mismatch: stats->status or
+ * moe_workspace_status MOE_ERR_INVALID).  Otherwise the histograms are not
+ * read.
+ */
+moe_status moe_load_stats_tiles(const int32_t* topk_idx, int64_t T, int32_t K, int32_t N,
+                                const int32_t* tile_counts, const int32_t* replica_slot,
+                                int32_t n_slots, int32_t* slot_idx, int32_t* counts, int32_t* offsets,
+                                int32_t* rank, moe_stats* stats, void* ws, size_t ws_bytes,
+                                moe_stream_t stream);
 
 /*
  * moe_replica_plan -- replica slots for the n_replicas hottest experts.
@@ -330,8 +378,9 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
  *    at a new address): do not call this entry point after a device reset.
  *  - All calls share the one array, which keeps the last call's contents.
  *    Every call first clears, on its stream, the part that must start at
- *    zero (the scan's control words and look-back flags, a few KB), so a
- *    call never depends on how the previous one ended.  Calls whose kernels
+ *    zero (the scan's control words, look-back flags and per-block count
+ *    words: at most about 1.2 MB), so a call never depends on how the
+ *    previous one ended.  Calls whose kernels
  *    overlap on the GPU -- different streams, or threads, using the same
  *    device -- race on the array: the caller must serialise them.
  * The load status of the call is in stats->status, as for moe_load_stats.
@@ -350,11 +399,12 @@ moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T, int32_t K,
  * (The calls that synchronise are this one and moe_selftest_wait_timeout.) */
 moe_status moe_workspace_status(void* ws, moe_stream_t stream);
 
-/* Self-test of the bounded device waits: runs the offsets pass's look-back
- * on a two-block problem where the flag it waits for is never set.  The wait
- * must give up after about one second, record the timeout and return, and the
- * CUDA context stays usable.  Returns MOE_ERR_TIMEOUT when the wait ran out as
- * designed (the expected result), MOE_OK if it did not.  Synchronises
+/* Self-test of the bounded device waits: runs each load-statistics kernel's
+ * wait for an earlier block (the look-back, and the read of earlier blocks'
+ * tagged counts) on a two-block problem whose first block never runs.  Each
+ * wait must give up after about one second, record the timeout and return,
+ * and the CUDA context stays usable.  Returns MOE_ERR_TIMEOUT when both waits
+ * ran out as designed (the expected result), MOE_OK if not.  Synchronises
  * `stream`; ws needs moe_workspace_bytes(4096, 1, 8, 8) bytes; the
  * workspace's error words are cleared afterwards. */
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, moe_stream_t stream);

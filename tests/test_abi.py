@@ -173,3 +173,34 @@ def test_capacity_limit_is_the_pages_rule(moe):
         assert moe.capacity_limit(T, K, N) == oracle.capacity_limit(T, K, N)
     assert L.moe_capacity_limit(-1, 8, 256) == -1 and L.moe_capacity_limit(16, 0, 256) == -1
     assert L.moe_capacity_limit(16, 8, 0) == -1
+
+
+def test_route_tiles_and_tile_stats_reject_bad_arguments(moe):
+    """The fused entry points validate on the host: missing buffers, a shape
+    the epilogue cannot select, fp32 inputs, misalignment, a short workspace.
+    (Every call here fails before any launch.)"""
+    L = moe._lib
+    ws = L.moe_workspace_bytes(64, 8, 256, 256)
+    cfg = _cfg(moe)
+    by = ctypes.byref
+    # no tile histogram buffer
+    assert L.moe_route_tiles(by(cfg), FAKE, FAKE, None, None, FAKE, FAKE, None, FAKE, ws, None) == 1
+    # no x: the fused path needs the gate
+    assert L.moe_route_tiles(by(cfg), None, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, ws, None) == 1
+    # K > 8, N = 512 and fp32 inputs have no epilogue selection
+    assert L.moe_route_tiles(by(_cfg(moe, K=16, n_groups=1)), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, ws,
+                             None) == 2
+    assert L.moe_route_tiles(by(_cfg(moe, N=512, n_groups=16)), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE,
+                             L.moe_workspace_bytes(64, 8, 512, 512), None) == 2
+    assert L.moe_route_tiles(by(_cfg(moe, in_dtype=0)), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, ws,
+                             None) == 2
+    assert L.moe_route_tiles(by(cfg), MISALIGNED, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, ws, None) == 1
+    assert L.moe_route_tiles(by(cfg), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, ws - 1, None) == 1
+    # load statistics from tile histograms
+    wsl = L.moe_workspace_bytes(64, 8, 256, 256)
+    assert L.moe_load_stats_tiles(FAKE, 64, 8, 256, None, None, 256, None, FAKE, FAKE, FAKE, None, FAKE, wsl,
+                                  None) == 1
+    assert L.moe_load_stats_tiles(FAKE, 64, 8, 256, FAKE, None, 288, None, FAKE, FAKE, FAKE, None, FAKE, wsl,
+                                  None) == 1  # replica slots without a replica map
+    assert L.moe_load_stats_tiles(FAKE, 64, 8, 256, FAKE, None, 256, None, FAKE, FAKE, FAKE, None, FAKE, wsl - 1,
+                                  None) == 1

@@ -65,7 +65,9 @@ def test_selection_unnormalised_and_topn(orc):
 
 
 @pytest.mark.parametrize("T,K,N,skew,R", [(5000, 8, 256, 0.0, 0), (5000, 8, 256, 1.1, 32), (513, 2, 8, 0.0, 0),
-                                           (131072, 8, 256, 1.1, 32), (4096, 8, 128, 0.5, 0)])
+                                           (131072, 8, 256, 1.1, 32), (4096, 8, 128, 0.5, 0),
+                                           (65536, 8, 128, 0.3, 16), (40961, 8, 256, 0.9, 0),
+                                           (327681, 8, 256, 0.2, 0)])
 def test_histogram_offsets_ranks_stats(orc, T, K, N, skew, R):
     idx = W.make_assignments(T, K, N, seed=T + K, skew=skew)
     slot_i, counts, offsets, rank, stats, ws = load_stats_gpu(idx.cuda(), T, K, N)

@@ -158,3 +158,24 @@ def test_route_with_gate_outside_the_tensor_core_shapes(orc, N, K, G, TG, fn):
     assert (err <= 1e-3 * np.abs(s_ref) + 1e-7).all()
     ri, rw = orc.select(to_np(s), inp["bias"].numpy(), K, G, TG, 2, True, 2.5)
     assert np.array_equal(to_np(idx), ri) and np.array_equal(to_np(w), rw)
+
+
+def test_load_stats_kernels_share_one_workspace(orc):
+    """Problems above and below the chain-free kernel's limit (~2.6M
+    assignments: look-back kernel vs tagged-count kernel, one and several
+    blocks) alternate on one workspace; each call's counts, offsets and
+    ranks equal the oracle's, so neither kernel's left-over words (look-back
+    flags, tagged counts, prefixes) are ever read as this call's."""
+    N, K = 64, 8
+    sizes = [400000, 16384, 100, 131072, 400000, 70000, 100, 16384]
+    moe = lib()
+    ws = moe.workspace(max(sizes), K, N)
+    for i, T in enumerate(sizes):
+        idx = W.make_assignments(T, K, N, seed=50 + i, device="cuda", skew=0.6)
+        slot, counts, offsets, rank, stats, _ = load_stats_gpu(idx, T, K, N, ws=ws)
+        c_ref, off_ref, _, rank_ref, _ = orc.positions(to_np(idx), N)
+        assert np.array_equal(to_np(counts), c_ref), T
+        assert np.array_equal(to_np(offsets), off_ref), T
+        assert np.array_equal(to_np(rank), rank_ref), T
+        assert_stats_close(moe.read_stats(stats), orc.load_stats(c_ref))
+    assert moe.moe_workspace_status(ws) == 0

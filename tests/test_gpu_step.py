@@ -72,3 +72,42 @@ def test_pipelined_with_host_copies_equals_serial():
         assert torch.equal(h, d.cpu())
     assert torch.equal(P.rows.view(torch.int16), S.rows.view(torch.int16))
     assert torch.equal(P.bias, S.bias)
+
+
+@pytest.mark.parametrize("name,T,steps,fused", [("metric", 2048, 6, False), ("softmax_dispatch", 1500, 5, False),
+                                                ("metric", 2048, 6, True), ("softmax_dispatch", 1500, 5, True)])
+def test_every_batch_with_combine_equals_serial(name, T, steps, fused):
+    """Each batch's indices, weights, offsets, counts and stats (copied to the
+    host on the routing stream right after its routing) and its combine
+    output (identity experts, on the caller's stream after its dispatch) are
+    the same in both schedules, for every batch: with the routing outputs
+    double-buffered, batch i+1's routing never overwrites what batch i's
+    dispatch and combine still read."""
+    wl = W.WORKLOADS[name].with_(T=T)
+    xs = [W.make_inputs(wl, device="cuda", seed=20 + j)["x"] for j in range(3)]
+    inp = W.make_inputs(wl, device="cuda", seed=19)
+    bias0 = inp["bias"] if inp["bias"] is not None else torch.zeros(wl.N, device="cuda")
+    got = {}
+    for pipelined in (False, True):
+        # the serial reference always takes the unfused path: both paths route identically
+        S = RoutingStep(wl, xs, inp["W"], bias0.clone(), inp["off"], "cuda", pipelined=pipelined,
+                        fused=fused and pipelined)
+        host, outs = [], []
+        for i in range(steps):
+            h = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in S.results(S.sets[0])]
+            o = torch.empty(wl.T, wl.d, dtype=xs[0].dtype, device="cuda")
+            S.step(host_out=h, combine_out=o)
+            host.append(h)
+            outs.append(o)
+        torch.cuda.synchronize()
+        got[pipelined] = (host, outs)
+    for i in range(steps):
+        for a, b in zip(got[False][0][i], got[True][0][i]):
+            assert torch.equal(a, b), i
+        assert torch.equal(got[False][1][i].view(torch.int16), got[True][1][i].view(torch.int16)), i
+        # identity experts with weights summing to the route scale: out = scale * x up to rounding
+        x = xs[i % len(xs)].float()
+        scale = wl.scale if wl.renorm else None
+        if scale is not None:
+            diff = (got[True][1][i].float() - scale * x).abs()
+            assert (diff <= (scale * x).abs() * 2.0 ** -6 + 1e-5).all(), i
