@@ -564,7 +564,8 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: 8 independent loads at a time
+    // 3. counts of all earlier blocks, per slot: 16 independent loads at a time
+    constexpr int PB = 16;
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false;
 #pragma unroll
@@ -573,13 +574,13 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         const int e = tid + j * LS_THREADS;
         if (e >= n_slots || b == 0) continue;
         uint64_t t0 = 0;
-        for (int q0 = 0; q0 < b; q0 += 8) {
-            uint64_t v[8];
+        for (int q0 = 0; q0 < b; q0 += PB) {
+            uint64_t v[PB];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
+            for (int u = 0; u < PB; ++u)
                 v[u] = q0 + u < b ? ld_relaxed_u64(agg64 + (int64_t)(q0 + u) * n_slots + e) : ((uint64_t)tag << 32);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < PB; ++u) {
                 // bounded re-poll of a word this call's block q0+u has not published yet
                 while ((uint32_t)(v[u] >> 32) != tag && !timed_out) {
                     if (t0 == 0) t0 = globaltimer();

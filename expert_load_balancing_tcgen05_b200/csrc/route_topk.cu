@@ -456,14 +456,15 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(SW_THREADS) route_select_warp_kernel(
+__global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
     const float* __restrict__ scores, const float* __restrict__ bias, int T, int K, int grouped, int topk_groups,
     int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     constexpr int N = 32 * EPL;
     constexpr int G = 32 / EPL;  // lanes per group of 32 experts
-    __shared__ float l_key[SW_THREADS / 32][32], l_s[SW_THREADS / 32][32];
+    __shared__ __align__(16) float l_key[SW_THREADS / 32][32];
+    __shared__ float l_s[SW_THREADS / 32][32];
     __shared__ int l_idx[SW_THREADS / 32][32];
-    __shared__ float o_s[SW_THREADS / 32][8];
+    __shared__ __align__(16) float o_s[SW_THREADS / 32][8];
     __shared__ int o_i[SW_THREADS / 32][8];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int e0 = lane * EPL;
@@ -473,9 +474,15 @@ __global__ void __launch_bounds__(SW_THREADS) route_select_warp_kernel(
     const int rounds = (K + 1) >> 1;
     const int warps = gridDim.x * (SW_THREADS / 32);
 
-    for (int64_t t = (int64_t)blockIdx.x * (SW_THREADS / 32) + wib; t < T; t += warps) {
+    // the next token's row is loaded while the current one is ranked
+    float nv[EPL];
+    int64_t t = (int64_t)blockIdx.x * (SW_THREADS / 32) + wib;
+    if (t < T) load_row<EPL>(scores + t * N, lane, N, nv);
+    for (; t < T; t += warps) {
         float sv[EPL], kv[EPL];
-        load_row<EPL>(scores + t * N, lane, N, sv);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) sv[i] = nv[i];
+        if (t + warps < T) load_row<EPL>(scores + (t + warps) * N, lane, N, nv);
 #pragma unroll
         for (int i = 0; i < EPL; ++i) kv[i] = __fadd_rn(sv[i], b[i]);
         // 1. the lane's two largest keys
@@ -543,9 +550,18 @@ __global__ void __launch_bounds__(SW_THREADS) route_select_warp_kernel(
             __syncwarp();
             const float kc = lane < total ? l_key[wib][lane] : -INFINITY;
             int rank = 0;
-            for (int c2 = 0; c2 < total; ++c2) {
-                const float k2 = l_key[wib][c2];
-                rank += (k2 > kc || (k2 == kc && c2 < lane)) ? 1 : 0;
+            // the whole list in broadcast vector reads, all independent
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (4 * q < total) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(&l_key[wib][4 * q]);
+                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c2 = 4 * q + u;
+                        rank += (c2 < total && (kk[u] > kc || (kk[u] == kc && c2 < lane))) ? 1 : 0;
+                    }
+                }
             }
             if (lane < total && rank < K) {
                 o_i[wib][rank] = l_idx[wib][lane];
@@ -575,8 +591,13 @@ __global__ void __launch_bounds__(SW_THREADS) route_select_warp_kernel(
         }
         // outputs: weights from the unbiased scores, summed in k order
         if (lane < K) {
-            float ssum = o_s[wib][0];
-            for (int k = 1; k < K; ++k) ssum = __fadd_rn(ssum, o_s[wib][k]);
+            const float4 s0 = *reinterpret_cast<const float4*>(&o_s[wib][0]);
+            const float4 s1 = *reinterpret_cast<const float4*>(&o_s[wib][4]);
+            const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            float ssum = ss[0];
+#pragma unroll
+            for (int k = 1; k < 8; ++k)
+                if (k < K) ssum = __fadd_rn(ssum, ss[k]);
             const float sk = o_s[wib][lane];
             const float wv = renorm ? __fdiv_rn(sk, ssum) : sk;
             topk_idx[t * K + lane] = o_i[wib][lane];
@@ -620,8 +641,10 @@ cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int
     const char* env = getenv("MOE_SELECT_KERNEL");  // "filtered": the thread-per-group kernel (measurement)
     const bool filtered = env != nullptr && env[0] == 'f';
     if (!filtered && select_warp_ok(N, K, n_groups, group_topn)) {
+        // one wave of resident blocks (three per SM at this kernel's registers); each warp
+        // walks its tokens with the next row's load in flight
         long long blocks = ((long long)T + SW_THREADS / 32 - 1) / (SW_THREADS / 32);
-        const long long cap = (long long)moe_host::sm_count() * 8;
+        const long long cap = (long long)moe_host::sm_count() * 3;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
         const int grouped = n_groups > 1 ? 1 : 0;
