@@ -131,7 +131,7 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------
-def make_step(wl, rank, dev, world, pipelined, fused=False):
+def make_step(wl, rank, dev, world, pipelined, fused=False, gate_ctas=None):
     """The routing step on this rank's batches (inputs drawn on the device).
     Consecutive steps alternate between two distinct token batches in
     different buffers, so that overlapped steps never share rows of x in L2."""
@@ -140,7 +140,7 @@ def make_step(wl, rank, dev, world, pipelined, fused=False):
     inp = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank)
     x2 = W.make_inputs(wl, device=dev, seed=wl.seed + 100 * rank + 50)["x"]
     return RoutingStep(wl, [inp["x"], x2], inp["W"], inp["bias"].clone(), inp["off"], dev, world=world,
-                       pipelined=pipelined, fused=fused)
+                       pipelined=pipelined, fused=fused, gate_max_ctas=gate_ctas if pipelined else None)
 
 
 def stage_bytes(wl):
@@ -202,13 +202,16 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[WORKLOAD_NAME]
     pipelined = not args.serial
-    P = make_step(wl, rank, dev, world, pipelined, fused=args.fused)
+    P = make_step(wl, rank, dev, world, pipelined, fused=args.fused, gate_ctas=args.gate_ctas)
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
+    # clocks are sampled from before the warm-up to after the timed region
+    sampler = ClockSampler(local_rank)
+    sampler.start()
     # warm-up (also ramps clocks) and a correctness status check
     w0 = time.time()
     n_warm = max(args.warmup, 3)
@@ -230,10 +233,8 @@ def run_ours(args, rank, world, local_rank):
             P.step()
         torch.cuda.synchronize()
 
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    # soak ~0.3 s so the sampler sees the loaded clock before and during timing
-    soak(0.3)
+    # soak ~0.6 s so the sampler sees the loaded clock before and during timing
+    soak(0.6)
 
     E = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     moe.moe_launch_count(reset=True)
@@ -249,12 +250,22 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     launches = moe.moe_launch_count()
     # keep the sampler running over a few more steps so short timed regions still get samples
-    soak(0.2)
+    soak(0.4)
     clocks = sampler.summarise(sampler.stop())
     ms = start.elapsed_time(stop)
     t_disp = statistics.mean(a.elapsed_time(b) for a, b in E)
     del P
     torch.cuda.empty_cache()
+    if args.timed_only:
+        # a sweep point: the timed region only (no serial stages, combine or end-to-end leg)
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        return {"metric": METRIC, "value": wl.T * args.steps * world / (ms_max / 1e3), "unit": UNIT,
+                "ms_per_step": ms_max / args.steps, "timed_only": True, "fused": args.fused,
+                "gate_ctas": args.gate_ctas, "dispatch_ms_in_timed_region": t_disp, "clocks": clocks} \
+            if rank == 0 else None
 
     # the serial schedule: per-stage times (route, load statistics + bias
     # step, dispatch), the combine loop and the end-to-end leg
@@ -302,7 +313,7 @@ def run_ours(args, rank, world, local_rank):
     # the device for the expert GEMMs.
     del S
     torch.cuda.empty_cache()
-    E2 = make_step(wl, rank, dev, world, pipelined, fused=args.fused)
+    E2 = make_step(wl, rank, dev, world, pipelined, fused=args.fused, gate_ctas=args.gate_ctas)
     x_host = E2.x.cpu().pin_memory()
     x_dev = [torch.empty_like(E2.x) for _ in range(2)]
     res_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in E2.results(E2.sets[0])]
@@ -921,6 +932,10 @@ def main():
     ap.add_argument("--report", action="store_true",
                     help="print the bias-balancing trajectory, the replica loads and per-workload GPU vs oracle "
                          "throughput (markdown)")
+    ap.add_argument("--gate-ctas", type=int, default=None,
+                    help="SM budget of the gate in the pipelined schedule (default: the step's own)")
+    ap.add_argument("--timed-only", action="store_true",
+                    help="print only the timed region's numbers (for sweeps; not the benchmark's full line)")
     ap.add_argument("--fused", action="store_true",
                     help="route through the fused path (selection and tile histograms in the gate's epilogue)")
     ap.add_argument("--serial", action="store_true",
@@ -953,7 +968,7 @@ def main():
     try:
         out = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and not args.timed_only:
                 out["cpu_baseline"] = cpu_baseline()
             print(json.dumps(out), flush=True)
     finally:

@@ -82,7 +82,7 @@ __device__ __forceinline__ int ld_volatile(const int32_t* p) { return *reinterpr
 // Each block takes the next ticket b and the assignments [b*2048, (b+1)*2048).
 //  1. slot of every assignment (replica remap), warp-private shared-memory
 //     histograms and the stable rank of each assignment inside its warp's
-//     chunk run (__match_any_sync: peers with the same slot, rank = peers
+//     chunk run (warp_slot_rank: peers with the same slot, rank = peers
 //     before me + what the warp saw earlier);
 //  2. per-slot prefix over the block's warps and the block's slot counts,
 //     published as the block aggregate (flag 1);
@@ -191,6 +191,33 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, bool tot_share
 
 constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
 
+// Place of each lane's assignment among the warp's assignments to the same
+// slot so far (the warp's running histogram `my`, in shared memory), in lane
+// order.  The lanes holding the same slot are found by one ballot per bit of
+// the slot (nbits = bits of n_slots - 1) instead of __match_any_sync, whose
+// cost grows with the number of distinct values; the lowest of them adds the
+// group's size to the histogram with one shared-memory atomic.  Lanes with
+// slot < 0 get an unused value.  Call with the whole warp, chunks in order;
+// the __syncwarp orders consecutive chunks' atomics on one slot.
+__device__ __forceinline__ int warp_slot_rank(int slot, int nbits, int32_t* my, int lane) {
+    unsigned peers = __ballot_sync(FULL, slot >= 0);
+    if (slot < 0) peers = ~peers;
+#pragma unroll
+    for (int bit = 0; bit < 11; ++bit) {
+        if (bit < nbits) {
+            const unsigned B = __ballot_sync(FULL, (slot >> bit) & 1);
+            peers &= ((slot >> bit) & 1) ? B : ~B;
+        }
+    }
+    const int before = __popc(peers & lanemask_lt());
+    const int leader = __ffs(peers) - 1;
+    int seen = 0;
+    if (slot >= 0 && lane == leader) seen = atomicAdd(my + slot, __popc(peers));
+    seen = __shfl_sync(FULL, seen, leader);
+    __syncwarp();
+    return seen + before;
+}
+
 // Block end: the last block to finish folds this call's error bits into the
 // sticky word and resets the control words for the next call.
 __device__ __forceinline__ void block_done(ScanCtl* ctl, int64_t nblk) {
@@ -243,6 +270,7 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
 
     // 1. slots, warp histograms, in-warp stable ranks (all loads issued first)
     int32_t* my = wh + warp * n_slots;
+    const int nbits = n_slots > 1 ? 32 - __clz(n_slots - 1) : 0;
     const int64_t base_a = b * LS_BLOCK + (int64_t)warp * (LS_CHUNKS * 32);
     int slot_r[LS_CHUNKS], rank_r[LS_CHUNKS];
 #pragma unroll
@@ -268,14 +296,8 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
             }
             if (slot_out != nullptr) slot_out[a] = slot;
         }
-        const unsigned peers = __match_any_sync(FULL, slot);
-        const int before = __popc(peers & lanemask_lt());
-        const int seen = (slot >= 0) ? my[slot] : 0;
-        __syncwarp();
-        if (slot >= 0 && before == 0) my[slot] = seen + __popc(peers);
-        __syncwarp();
+        rank_r[j] = warp_slot_rank(slot, nbits, my, lane);
         slot_r[j] = slot;
-        rank_r[j] = seen + before;
     }
     if (bad) atomicOr(&ctl->err, 2);
     __syncthreads();
@@ -409,37 +431,41 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
 // C chunks of 32 (one wave of at most ~320 blocks):
 //  1. slots, warp histograms and in-warp stable ranks, as above;
 //  2. per-slot prefix over the block's warps; the block's per-slot counts are
-//     published as 64-bit words whose high half carries this call's tag
-//     (bit 31 | epoch), so a word is its own ready flag: no separate flag and
-//     no fence on the normal path (a word without the tag -- zero, an older
-//     call's, or another layout's int32 data, which never has bit 31 in that
-//     half -- reads as "not yet");
-//  3. each block sums, per slot, the words of ALL earlier blocks (independent
-//     loads, a bounded re-poll of any word not yet tagged): the count of every
-//     earlier assignment in that slot, without waiting on inclusive prefixes;
+//     published as 32-bit words with bit 31 set, so a word is its own ready
+//     flag: no separate flag and no fence on the normal path (a word without
+//     bit 31 -- zero, or the look-back kernel's counts, which never have it
+//     -- reads as "not yet");
+//  3. each block sums, per slot, the words of ALL earlier blocks (32
+//     independent loads at a time, a bounded re-poll of any word not yet
+//     ready): the count of every earlier assignment in that slot, without
+//     waiting on inclusive prefixes;
 //  4. rank = earlier blocks + earlier warps + within the warp;
 //  5. the last block's sums plus its own counts are the totals: counts,
-//     offsets, statistics.  The last block to finish advances the epoch.
+//     offsets, statistics.  The last block to finish -- no block reads the
+//     words any more -- clears this call's words, so no ready word outlives
+//     its call, and resets the control words.
 // A one-block problem shares nothing with other blocks: it publishes nothing,
 // waits for nothing and leaves the control words untouched (error bits go to
 // the sticky word directly).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+
+constexpr uint32_t WORD_READY = 0x80000000u;  // a published per-block count: bit 31 | count
 
 template <int C>
 __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     const int32_t* __restrict__ idx, int64_t A, int K, int N, const int32_t* __restrict__ replica_slot,
     int n_slots, int32_t* __restrict__ slot_out, int32_t* __restrict__ rank_out, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, moe_stats* stats, const double* __restrict__ hs_partial, int hs_blocks,
-    int64_t T, ScanCtl* ctl, uint64_t* agg64, int nblk, int block_base, const int32_t* __restrict__ tile_counts) {
+    int64_t T, ScanCtl* ctl, uint32_t* aggw, int nblk, int block_base, const int32_t* __restrict__ tile_counts) {
     constexpr int BPB = LS_WARPS * C * 32;
     extern __shared__ int32_t sm_dyn[];
     int32_t* wh = sm_dyn;                       // [LS_WARPS][n_slots]
@@ -459,8 +485,6 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         const int64_t a = base_a + j * 32 + lane;
         slot_r[j] = a < A ? __ldg(idx + a) : -1;
     }
-    const uint32_t tag = multi ? (0x80000000u | (uint32_t)ld_volatile(reinterpret_cast<const int32_t*>(&ctl->epoch)))
-                               : 0u;
     if (tid == 0) s_err = 0;
     for (int i = tid; i < LS_WARPS * n_slots; i += LS_THREADS) wh[i] = 0;
     // the gate epilogue's per-tile histograms (tiles of 128 tokens, aligned to
@@ -495,7 +519,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                         if (e < N) c += __ldg(tq + src) + (has_rep ? 0 : __ldg(tq + N + src));
                         else c += __ldg(tq + N + src);
                     }
-                if (b < nblk - 1) st_relaxed_u64(agg64 + (int64_t)b * n_slots + e, ((uint64_t)tag << 32) | (uint32_t)c);
+                if (b < nblk - 1) st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (uint32_t)c);
             }
             tc_agg[j] = c;
         }
@@ -504,6 +528,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
 
     // 1. slots, warp histograms, in-warp stable ranks
     int32_t* my = wh + warp * n_slots;
+    const int nbits = n_slots > 1 ? 32 - __clz(n_slots - 1) : 0;
     int bad = 0;
 #pragma unroll
     for (int j = 0; j < C; ++j) {
@@ -522,14 +547,8 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
             }
             if (slot_out != nullptr) slot_out[a] = slot;
         }
-        const unsigned peers = __match_any_sync(FULL, slot);
-        const int before = __popc(peers & lanemask_lt());
-        const int seen = (slot >= 0) ? my[slot] : 0;
-        __syncwarp();
-        if (slot >= 0 && before == 0) my[slot] = seen + __popc(peers);
-        __syncwarp();
+        rank_r[j] = warp_slot_rank(slot, nbits, my, lane);
         slot_r[j] = slot;
-        rank_r[j] = seen + before;
     }
     if (__any_sync(FULL, bad) && lane == 0) atomicOr(&s_err, 2);
     __syncthreads();
@@ -559,13 +578,13 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
             if (pre_published) {
                 if (tc_agg[j] != run) atomicOr(&s_err, 2);  // the tile histograms do not match the indices
             } else if (multi && b < nblk - 1) {
-                st_relaxed_u64(agg64 + (int64_t)b * n_slots + e, ((uint64_t)tag << 32) | (uint32_t)run);
+                st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (uint32_t)run);
             }
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: 16 independent loads at a time
-    constexpr int PB = 16;
+    // 3. counts of all earlier blocks, per slot: 32 independent loads at a time
+    constexpr int PB = 32;
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false;
 #pragma unroll
@@ -575,20 +594,20 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         if (e >= n_slots || b == 0) continue;
         uint64_t t0 = 0;
         for (int q0 = 0; q0 < b; q0 += PB) {
-            uint64_t v[PB];
+            uint32_t v[PB];
 #pragma unroll
             for (int u = 0; u < PB; ++u)
-                v[u] = q0 + u < b ? ld_relaxed_u64(agg64 + (int64_t)(q0 + u) * n_slots + e) : ((uint64_t)tag << 32);
+                v[u] = q0 + u < b ? ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e) : WORD_READY;
 #pragma unroll
             for (int u = 0; u < PB; ++u) {
                 // bounded re-poll of a word this call's block q0+u has not published yet
-                while ((uint32_t)(v[u] >> 32) != tag && !timed_out) {
+                while (!(v[u] & WORD_READY) && !timed_out) {
                     if (t0 == 0) t0 = globaltimer();
                     else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
                     __nanosleep(64);
-                    v[u] = ld_relaxed_u64(agg64 + (int64_t)(q0 + u) * n_slots + e);
+                    v[u] = ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e);
                 }
-                excl[j] += (uint32_t)(v[u] >> 32) == tag ? (int)(uint32_t)v[u] : 0;
+                excl[j] += (v[u] & WORD_READY) ? (int)(v[u] & ~WORD_READY) : 0;
             }
         }
     }
@@ -625,7 +644,25 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         __syncthreads();
         if (tid == 0 && (s_err & ~blk_err)) atomicOr(&ctl->err, s_err & ~blk_err);  // timeouts, histogram mismatch
         __syncthreads();
-        block_done(ctl, nblk);
+        // the last block to finish clears this call's count words (no block
+        // reads them any more) and resets the control words
+        __shared__ int s_last;
+        if (tid == 0) {
+            __threadfence();
+            s_last = atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int64_t i = tid; i < (int64_t)(nblk - 1) * n_slots; i += LS_THREADS) aggw[i] = 0u;
+            if (tid == 0) {
+                ctl->sticky |= ctl->err;
+                ctl->err = 0;
+                ctl->done = 0;
+                ctl->ticket = 0;
+                ctl->epoch = ctl->epoch + 1;
+            }
+        }
     } else if (tid == 0 && s_err != 0) {
         atomicOr(&ctl->sticky, s_err);  // read and cleared by moe_workspace_status
     }
@@ -768,7 +805,7 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
     const int64_t nb2 = (A + (int64_t)LS_THREADS * chunks - 1) / ((int64_t)LS_THREADS * chunks);
     if (nb2 <= V2_MAX_BLOCKS) {
         const int nb = nb2 < 1 ? 1 : (int)nb2;
-        uint64_t* agg64 = reinterpret_cast<uint64_t*>(agg);  // the agg and pre regions hold 8 bytes per cell
+        uint32_t* aggw = reinterpret_cast<uint32_t*>(agg);  // one ready-flagged count word per (block, slot)
         auto kern = chunks == 8 ? load_stats_v2_kernel<8> : (chunks == 16 ? load_stats_v2_kernel<16>
                                                                           : load_stats_v2_kernel<32>);
         if (lsm > 48 * 1024) {
@@ -779,7 +816,7 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
         const int bpb = LS_THREADS * chunks;
         const bool tiles_ok = tile_counts != nullptr && bpb % K == 0 && (bpb / K) % 128 == 0;
         kern<<<nb, LS_THREADS, lsm, st>>>(idx, A, K, N, replica_slot, n_slots, slot_idx, rank, counts, offsets, stats,
-                                          part, HS_BLOCKS, T, ctl, agg64, nb, 0, tiles_ok ? tile_counts : nullptr);
+                                          part, HS_BLOCKS, T, ctl, aggw, nb, 0, tiles_ok ? tile_counts : nullptr);
         moe_host::note_launch();
         return cudaGetLastError();
     }
@@ -796,8 +833,8 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
 
 // Self-test of the bounded waits of both load-statistics kernels: a
 // two-block problem (no assignments, 8 slots) of which only the second block
-// is launched, so block 0 never publishes (its look-back flag, or its tagged
-// counts, never appear).  Each probe block must give up after the wait
+// is launched, so block 0 never publishes (its look-back flag, or its ready
+// count words, never appear).  Each probe block must give up after the wait
 // limit, set the timeout bit and finish.  Returns the error bits of the two
 // probes and'ed (bit 0 set only if both waits ran out).
 cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t st) {
@@ -807,7 +844,8 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
     int32_t bits = ~0;
     for (int probe = 0; probe < 2; ++probe) {
         // ticket, finished count and error words start at zero; the epoch
-        // stays, so flags and tagged counts left by earlier calls are stale
+        // stays, so flags left by earlier calls are stale (count words are
+        // cleared by every call's last block)
         cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
         if (e != cudaSuccess) return e;
         const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8;
@@ -819,7 +857,7 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
         else
             load_stats_v2_kernel<8><<<1, LS_THREADS, smem, st>>>(
                 nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,
-                reinterpret_cast<uint64_t*>(w + L.agg), /*nblk=*/2, /*block_base=*/1, nullptr);
+                reinterpret_cast<uint32_t*>(w + L.agg), /*nblk=*/2, /*block_base=*/1, nullptr);
         moe_host::note_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ScanCtl h;

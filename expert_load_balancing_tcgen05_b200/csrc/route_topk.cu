@@ -436,13 +436,15 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
 //      integer images of the keys).  At least ceil(K/2) kept lanes hold two
 //      keys >= theta, so at least K kept keys are >= theta and the K best
 //      keys are all >= theta;
-//   4. the survivors (kept keys >= theta; typically K to K+4) are written to
-//      a per-warp shared list in expert order, one per lane, and each lane
-//      ranks its survivor against the others (rank = how many beat it by key
-//      desc, list position asc = index asc); survivors of rank < K are
-//      placed at their rank; lanes 0..K-1 write the outputs, the weights
-//      from the unbiased scores summed in k order.  A token with more than
-//      32 survivors takes K rounds of a warp argmax instead.
+//   4. the survivors (kept keys >= theta; typically K to K+4) are moved
+//      through a per-warp shared list, in expert order, to one per lane;
+//   5. K rounds of a warp max-reduction (redux.sync) over the survivors'
+//      order-preserving key images pick the choices in (key desc, index asc)
+//      order -- among equal keys the lowest lane, which holds the lowest
+//      index; lane k takes the k-th choice, and lanes 0..K-1 write the
+//      outputs, the weights from the unbiased scores summed in k order.  A
+//      token with more than 32 survivors takes K rounds of a warp argmax over
+//      its survivors in registers instead.
 // The result is the plain definition's: the survivors contain the K best
 // kept keys and the ranking is the (key desc, index asc) order.
 // ---------------------------------------------------------------------------
@@ -461,11 +463,8 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
     int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     constexpr int N = 32 * EPL;
     constexpr int G = 32 / EPL;  // lanes per group of 32 experts
-    __shared__ __align__(16) float l_key[SW_THREADS / 32][32];
-    __shared__ float l_s[SW_THREADS / 32][32];
+    __shared__ float l_key[SW_THREADS / 32][32], l_s[SW_THREADS / 32][32];
     __shared__ int l_idx[SW_THREADS / 32][32];
-    __shared__ __align__(16) float o_s[SW_THREADS / 32][8];
-    __shared__ int o_i[SW_THREADS / 32][8];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int e0 = lane * EPL;
     float b[EPL];
@@ -519,7 +518,7 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
             th_u = __reduce_max_sync(FULL, u2);
             if (u2 == th_u) u2 = 0u;
         }
-        // 4. survivors, compacted in expert order
+        // 4. survivors, compacted in expert order, one per lane
         unsigned m = 0;
         if (kept) {
 #pragma unroll
@@ -527,6 +526,8 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
         }
         const int cnt = __popc(m);
         const int total = __reduce_add_sync(FULL, (unsigned)cnt);
+        int my_i = 0;
+        float my_s = 0.f;
         if (total <= 32) {
             int off = cnt;
 #pragma unroll
@@ -535,43 +536,35 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
                 if (lane >= o) off += y;
             }
             off -= cnt;
-            while (m) {
-                const int i = __ffs(m) - 1;
-                m &= m - 1;
 #pragma unroll
-                for (int q = 0; q < EPL; ++q)
-                    if (q == i) {
-                        l_key[wib][off] = kv[q];
-                        l_s[wib][off] = sv[q];
-                    }
-                l_idx[wib][off] = e0 + i;
-                ++off;
-            }
-            __syncwarp();
-            const float kc = lane < total ? l_key[wib][lane] : -INFINITY;
-            int rank = 0;
-            // the whole list in broadcast vector reads, all independent
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                if (4 * q < total) {
-                    const float4 k4 = *reinterpret_cast<const float4*>(&l_key[wib][4 * q]);
-                    const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c2 = 4 * q + u;
-                        rank += (c2 < total && (kk[u] > kc || (kk[u] == kc && c2 < lane))) ? 1 : 0;
-                    }
+            for (int i = 0; i < EPL; ++i) {  // predicated stores, no branches
+                if ((m >> i) & 1u) {
+                    l_key[wib][off] = kv[i];
+                    l_s[wib][off] = sv[i];
+                    l_idx[wib][off] = e0 + i;
                 }
-            }
-            if (lane < total && rank < K) {
-                o_i[wib][rank] = l_idx[wib][lane];
-                o_s[wib][rank] = l_s[wib][lane];
+                off += (int)((m >> i) & 1u);
             }
             __syncwarp();
+            const bool has = lane < total;
+            uint32_t uk = has ? ord_key(l_key[wib][lane]) : 0u;
+            const int ci = has ? l_idx[wib][lane] : 0;
+            const float cs = has ? l_s[wib][lane] : 0.f;
+            __syncwarp();
+            // 5. K rounds: the largest key; among equal keys the lowest lane,
+            //    which holds the lowest index (the list is in expert order)
+            int winner_k = 0;
+            for (int k = 0; k < K; ++k) {
+                const uint32_t mx = __reduce_max_sync(FULL, uk);
+                const unsigned tie = __ballot_sync(FULL, uk == mx && has);
+                const int w = __ffs(tie) - 1;
+                if (lane == w) uk = 0u;
+                if (lane == k) winner_k = w;
+            }
+            my_i = __shfl_sync(FULL, ci, winner_k);
+            my_s = __shfl_sync(FULL, cs, winner_k);
         } else {
             // more survivors than lanes: K rounds of a warp argmax over them
-            int my_i = 0;
-            float my_s = 0.f;
             for (int k = 0; k < K; ++k) {
                 float bk = -INFINITY, bs = 0.f;
                 int bi = 0x7fffffff;
@@ -586,24 +579,21 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
                 if (lane == owner) m &= ~(1u << (wi - e0));
                 if (lane == k) { my_i = wi; my_s = ws; }
             }
-            if (lane < K) { o_i[wib][lane] = my_i; o_s[wib][lane] = my_s; }
-            __syncwarp();
         }
-        // outputs: weights from the unbiased scores, summed in k order
-        if (lane < K) {
-            const float4 s0 = *reinterpret_cast<const float4*>(&o_s[wib][0]);
-            const float4 s1 = *reinterpret_cast<const float4*>(&o_s[wib][4]);
-            const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-            float ssum = ss[0];
+        // outputs: lane k holds the k-th choice; weights from the unbiased
+        // scores summed in k order
+        float sk[8];
 #pragma unroll
-            for (int k = 1; k < 8; ++k)
-                if (k < K) ssum = __fadd_rn(ssum, ss[k]);
-            const float sk = o_s[wib][lane];
-            const float wv = renorm ? __fdiv_rn(sk, ssum) : sk;
-            topk_idx[t * K + lane] = o_i[wib][lane];
+        for (int k = 0; k < 8; ++k) sk[k] = __shfl_sync(FULL, my_s, k);
+        float ssum = sk[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k)
+            if (k < K) ssum = __fadd_rn(ssum, sk[k]);
+        if (lane < K) {
+            const float wv = renorm ? __fdiv_rn(my_s, ssum) : my_s;
+            topk_idx[t * K + lane] = my_i;
             topk_w[t * K + lane] = __fmul_rn(wv, route_scale);
         }
-        __syncwarp();
     }
 }
 
