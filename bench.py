@@ -6,10 +6,13 @@
 One step = one pass of the routing path over one batch of the throughput
 workload (T=16384 tokens, d=7168, N=256 experts, K=8, sigmoid scores, 8 groups
 keep 4, bias, weights x2.5):
-  moe_route       gate GEMM (tcgen05) + sigmoid + group-limited top-K + weights
-  moe_load_stats  histogram, look-back offsets, in-expert ranks, load stats
-  moe_bias_update sign-rule bias step
-  moe_dispatch    bf16 rows into the expert-contiguous buffer (+ positions)
+  moe_route_tiles      gate GEMM (tcgen05) + sigmoid + group-limited top-K +
+                       weights + per-tile expert histograms, all in the GEMM
+                       epilogue (no scores in memory)
+  moe_load_stats_tiles histogram, offsets, in-expert ranks, load stats
+  moe_bias_update      sign-rule bias step
+  moe_dispatch         bf16 rows into the expert-contiguous buffer (+ positions)
+(--unfused: moe_route writing the scores, the selection kernel, moe_load_stats.)
 Combine is timed in its own loop (identity experts: it gathers the
 dispatched rows back) and reported under "stages".
 
@@ -131,7 +134,7 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------
-def make_step(wl, rank, dev, world, pipelined, fused=False, gate_ctas=None):
+def make_step(wl, rank, dev, world, pipelined, fused=None, gate_ctas=None):
     """The routing step on this rank's batches (inputs drawn on the device).
     Consecutive steps alternate between two distinct token batches in
     different buffers, so that overlapped steps never share rows of x in L2."""
@@ -143,10 +146,27 @@ def make_step(wl, rank, dev, world, pipelined, fused=False, gate_ctas=None):
                        pipelined=pipelined, fused=fused, gate_max_ctas=gate_ctas if pipelined else None)
 
 
-def stage_bytes(wl):
-    """Algorithmic bytes / flops per launch (per batch of T tokens)."""
+def routing_path(args):
+    """None (the step's default: the fused path where the epilogue can select), or False with --unfused."""
+    return False if args.unfused else None
+
+
+def stage_bytes(wl, fused=False):
+    """Algorithmic bytes / flops per launch (per batch of T tokens).  The
+    fused path keeps the scores on chip: its gate writes the choices (and the
+    tile histograms) instead of the scores, and there is no separate
+    selection stage reading them back."""
     T, d, N, K = wl.T, wl.d, wl.N, wl.K
     A = T * K
+    if fused:
+        tiles = (T + 127) // 128 * 2 * N * 4
+        return {
+            "gate": {"bytes": T * d * 2 + N * d * 2 + A * 8 + tiles, "flops": 2 * T * d * N},
+            "topk": {"bytes": 0},
+            "hist": {"bytes": A * 4 * 2 + A * 4 + tiles + (N + 1) * 4 * 2},
+            "dispatch": {"bytes": T * d * 2 + A * d * 2 + A * 12},
+            "combine": {"bytes": A * d * 2 + A * 8 + T * d * 2},
+        }
     return {
         "gate": {"bytes": T * d * 2 + N * d * 2 + T * N * 4, "flops": 2 * T * d * N},
         "topk": {"bytes": T * N * 4 + N * 4 + A * 8},
@@ -156,13 +176,13 @@ def stage_bytes(wl):
     }
 
 
-def pipeline_roofline_us(wl, hbm_gbs, tflops, overlapped=False):
+def pipeline_roofline_us(wl, hbm_gbs, tflops, overlapped=False, fused=False):
     """Serial schedule: the stages one after another, each at the slower of
     its HBM and tensor bounds.  Overlapped schedule (routing of the next
     batch beside the dispatch): all stages share HBM, so the bound is the
     step's total bytes over HBM bandwidth, or the gate's tensor time if that
     is longer."""
-    b = stage_bytes(wl)
+    b = stage_bytes(wl, fused)
     stages = ("gate", "topk", "hist", "dispatch")
     if overlapped:
         tb = sum(b[k]["bytes"] for k in stages) / (hbm_gbs * 1e9)
@@ -202,7 +222,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[WORKLOAD_NAME]
     pipelined = not args.serial
-    P = make_step(wl, rank, dev, world, pipelined, fused=args.fused, gate_ctas=args.gate_ctas)
+    P = make_step(wl, rank, dev, world, pipelined, fused=routing_path(args), gate_ctas=args.gate_ctas)
+    P_fused = P.fused
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
 
     def barrier():
@@ -263,13 +284,13 @@ def run_ours(args, rank, world, local_rank):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_max = float(t.item())
         return {"metric": METRIC, "value": wl.T * args.steps * world / (ms_max / 1e3), "unit": UNIT,
-                "ms_per_step": ms_max / args.steps, "timed_only": True, "fused": args.fused,
+                "ms_per_step": ms_max / args.steps, "timed_only": True, "fused": not args.unfused,
                 "gate_ctas": args.gate_ctas, "dispatch_ms_in_timed_region": t_disp, "clocks": clocks} \
             if rank == 0 else None
 
     # the serial schedule: per-stage times (route, load statistics + bias
     # step, dispatch), the combine loop and the end-to-end leg
-    S = make_step(wl, rank, dev, world, pipelined=False, fused=args.fused)
+    S = make_step(wl, rank, dev, world, pipelined=False, fused=routing_path(args))
     for _ in range(3):
         S.step()
     n_stage = max(3, min(args.steps, 50))
@@ -313,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
     # the device for the expert GEMMs.
     del S
     torch.cuda.empty_cache()
-    E2 = make_step(wl, rank, dev, world, pipelined, fused=args.fused, gate_ctas=args.gate_ctas)
+    E2 = make_step(wl, rank, dev, world, pipelined, fused=routing_path(args), gate_ctas=args.gate_ctas)
     x_host = E2.x.cpu().pin_memory()
     x_dev = [torch.empty_like(E2.x) for _ in range(2)]
     res_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in E2.results(E2.sets[0])]
@@ -351,11 +372,11 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = wl.T * e2e_steps * world / (float(te.item()) / 1e3)
 
-    b = stage_bytes(wl)
+    b = stage_bytes(wl, fused=P_fused)
     disp_bytes = b["dispatch"]["bytes"]
     achieved = disp_bytes / (t_disp / 1e3) / 1e9
     traffic = _traffic_for("dispatch_combine.cu", "dispatch_metric_dram.json")
-    roof_us = pipeline_roofline_us(wl, hbm, tf_burst, overlapped=pipelined)
+    roof_us = pipeline_roofline_us(wl, hbm, tf_burst, overlapped=pipelined, fused=P_fused)
     ms_step = ms_max / args.steps
 
     out = None
@@ -365,7 +386,7 @@ def run_ours(args, rank, world, local_rank):
                     f"{PIPELINED_GATE_CTAS} SMs, selection, load statistics, bias step) on a high-priority stream beside "
                     "the dispatch of batch i") if pipelined else "serial: one call after another on one stream"
         schedule += ("; routing through the fused path (selection and per-tile histograms in the gate's epilogue, "
-                     "no scores in memory; statistics from the tile histograms)") if args.fused else \
+                     "no scores in memory; statistics from the tile histograms)") if not args.unfused else \
             "; routing through the gate's scores epilogue and the selection kernel"
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -393,6 +414,8 @@ def run_ours(args, rank, world, local_rank):
                 "dispatch_ms_in_timed_region": t_disp,
                 "combine_ms": t_comb,
                 "gate_topk_gbs_equiv": (b["gate"]["bytes"] + b["topk"]["bytes"]) / (t_route / 1e3) / 1e9,
+                "routing_path": "fused (moe_route_tiles + moe_load_stats_tiles)" if P_fused else
+                                "scores (moe_route + moe_load_stats)",
                 "gate_tflops_lower_bound": b["gate"]["flops"] / (t_route / 1e3) / 1e12,
                 "dispatch_gbs_serial": disp_bytes / (t_disp_serial / 1e3) / 1e9,
                 "combine_gbs": b["combine"]["bytes"] / (t_comb / 1e3) / 1e9,
@@ -936,8 +959,9 @@ def main():
                     help="SM budget of the gate in the pipelined schedule (default: the step's own)")
     ap.add_argument("--timed-only", action="store_true",
                     help="print only the timed region's numbers (for sweeps; not the benchmark's full line)")
-    ap.add_argument("--fused", action="store_true",
-                    help="route through the fused path (selection and tile histograms in the gate's epilogue)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="route through the gate's scores epilogue and the selection kernel instead of the fused "
+                         "path (selection and tile histograms in the gate's epilogue, the default)")
     ap.add_argument("--serial", action="store_true",
                     help="time the serial schedule (one call after another) instead of the pipelined one")
     args = ap.parse_args()

@@ -93,17 +93,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-// L2 prefetch of a tile of x a few k-steps ahead of its load into the ring
-// (a hint: nothing waits on it), so the ring's loads find it in L2 when HBM
-// is busy.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-constexpr int PF_KSTEPS_DEFAULT = 8;  // prefetch distance in k-steps (64 columns each); 0 = none
-
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle,
 // 8-row core-matrix groups 1024 bytes apart (SBO), sm_100 descriptor version.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
@@ -349,7 +338,7 @@ __device__ __forceinline__ void flush_tile_hist(const Epi& p, const Xch& x, int6
 template <int BN, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                              const __grid_constant__ CUtensorMap tmB, int d,
-                                                             const Epi p, int32_t* err, int num_tiles, int pf) {
+                                                             const Epi p, int32_t* err, int num_tiles) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -405,18 +394,9 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            // prefetch the first k-steps of this CTA's first tile
-            for (int kb = 0; kb < pf && kb < num_kb && (int)blockIdx.x < num_tiles; ++kb)
-                tma_prefetch_2d(&tmA, kb * BK, (int)blockIdx.x * BM);
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    // x tile pf k-steps ahead (continuing into this CTA's next tile)
-                    if (pf > 0) {
-                        const int kp = kb + pf;
-                        const int tp = kp < num_kb ? tile : tile + (int)gridDim.x;
-                        if (tp < num_tiles) tma_prefetch_2d(&tmA, (kp < num_kb ? kp : kp - num_kb) * BK, tp * BM);
-                    }
                     if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
                     mbar_expect_tx(full0 + 8 * s, C::STAGE_BYTES);
                     tma_load_2d(smem_u32(sA + (size_t)s * A_STAGE_BYTES), &tmA, kb * BK, tile * BM, full0 + 8 * s);
@@ -580,7 +560,7 @@ __device__ __forceinline__ constexpr uint32_t idesc_pair() {
 template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gate_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int d,
-                        const Epi p, int32_t* err, int num_pairs, int pf) {
+                        const Epi p, int32_t* err, int num_pairs) {
     constexpr int BN = 256, STAGES = PAIR_STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -638,19 +618,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int kb = 0; kb < pf && kb < num_kb && cluster < num_pairs; ++kb)
-                tma_prefetch_2d(&tmA, kb * BK, cluster * 2 * BM + (int)rank * BM);
             for (int tp = cluster; tp < num_pairs && ok; tp += nclusters) {
                 const int m0 = tp * 2 * BM + (int)rank * BM;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    // this CTA's x rows pf k-steps ahead (continuing into its next tile)
-                    if (pf > 0) {
-                        const int kp = kb + pf;
-                        const int tq = kp < num_kb ? tp : tp + nclusters;
-                        if (tq < num_pairs)
-                            tma_prefetch_2d(&tmA, (kp < num_kb ? kp : kp - num_kb) * BK, tq * 2 * BM + (int)rank * BM);
-                    }
                     if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
                     const uint32_t fb = map_to(full0 + 8 * s, 0);
                     if (leader) mbar_expect_tx(full0 + 8 * s, 2 * PAIR_STAGE_BYTES);
@@ -772,14 +743,6 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t col
 
 bool gate_tc_supported(int N) { return N == 64 || N == 128 || N == 256; }
 
-// L2 prefetch distance of the producers in k-steps (environment variable
-// MOE_GATE_PREFETCH overrides it; 0 turns the prefetch off)
-static int prefetch_ksteps() {
-    const char* e = getenv("MOE_GATE_PREFETCH");
-    if (e != nullptr && e[0] >= '0' && e[0] <= '9') return atoi(e);
-    return tc::PF_KSTEPS_DEFAULT;
-}
-
 // The epilogue can select when the groups are whole 32-column chunks (or
 // there is one group) and K fits its 8-entry list.
 bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn) {
@@ -801,7 +764,7 @@ static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const
     if (max_ctas > 0 && clusters > max_ctas / 2) clusters = max_ctas / 2;
     if (clusters > num_pairs) clusters = num_pairs;
     if (clusters < 1) clusters = 1;
-    kern<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs, prefetch_ksteps());
+    kern<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);
     moe_host::note_launch();
     return cudaGetLastError();
 }
@@ -820,7 +783,7 @@ static cudaError_t launch_bn(const void* x, const void* W, int T, int d, const t
     if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
     if (grid > num_tiles) grid = num_tiles;
     if (grid < 1) grid = 1;
-    kern<<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles, prefetch_ksteps());
+    kern<<<grid, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_tiles);
     moe_host::note_launch();
     return cudaGetLastError();
 }

@@ -197,8 +197,9 @@ constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
 // the slot (nbits = bits of n_slots - 1) instead of __match_any_sync, whose
 // cost grows with the number of distinct values; the lowest of them adds the
 // group's size to the histogram with one shared-memory atomic.  Lanes with
-// slot < 0 get an unused value.  Call with the whole warp, chunks in order;
-// the __syncwarp orders consecutive chunks' atomics on one slot.
+// slot < 0 get an unused value.  Call with the whole warp, chunks in order:
+// the leader's atomic returns before the warp-wide shuffle of its result, so
+// a later chunk's atomic on the same slot always sees it.
 __device__ __forceinline__ int warp_slot_rank(int slot, int nbits, int32_t* my, int lane) {
     unsigned peers = __ballot_sync(FULL, slot >= 0);
     if (slot < 0) peers = ~peers;
@@ -214,7 +215,6 @@ __device__ __forceinline__ int warp_slot_rank(int slot, int nbits, int32_t* my, 
     int seen = 0;
     if (slot >= 0 && lane == leader) seen = atomicAdd(my + slot, __popc(peers));
     seen = __shfl_sync(FULL, seen, leader);
-    __syncwarp();
     return seen + before;
 }
 
@@ -294,7 +294,6 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
                 if (r >= 0 && ((a / K) & 1)) slot = r;
                 if (slot >= n_slots) { bad = 1; slot = -1; }
             }
-            if (slot_out != nullptr) slot_out[a] = slot;
         }
         rank_r[j] = warp_slot_rank(slot, nbits, my, lane);
         slot_r[j] = slot;
@@ -404,11 +403,15 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
     __syncthreads();
     if (tid == 0 && b > 0) st_release_u32(flags + b, tag | FLAG_PREFIX);
 
-    // 4. in-expert ranks
+    // 4. in-expert ranks (and the slots, stored here rather than in the
+    //    histogram loop so that no store sits between its chunks)
 #pragma unroll
     for (int j = 0; j < LS_CHUNKS; ++j) {
         const int64_t a = base_a + j * 32 + lane;
-        if (a < A) rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+        if (a < A) {
+            rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+            if (slot_out != nullptr) slot_out[a] = slot_r[j];
+        }
     }
 
     // 5. the block with the last ticket holds the totals in its inclusive
@@ -458,7 +461,22 @@ __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-constexpr uint32_t WORD_READY = 0x80000000u;  // a published per-block count: bit 31 | count
+constexpr uint32_t WORD_READY = 0x80000000u;  // a published per-block count: bit 31 | bit 30 | count
+constexpr uint32_t WORD_BAD = 0x40000000u;    // the publishing block saw an expert id out of range
+constexpr uint32_t WORD_COUNT = 0x3fffffffu;
+
+__device__ __forceinline__ uint4 ld_relaxed_v4(const uint32_t* p) {
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+// Row stride (in words) of the per-slot count words: one word per block,
+// rounded up to whole 16-byte vectors.
+__host__ __device__ __forceinline__ int word_stride(int nblk) { return (nblk + 3) & ~3; }
 
 template <int C>
 __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
@@ -476,6 +494,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = block_base + (int)blockIdx.x;  // block_base > 0 only in the bounded-wait self-test
     const bool multi = nblk > 1;
+    const int wstride = word_stride(nblk);  // count words: aggw[slot * wstride + block]
 
     // the loads first: expert ids of this warp's chunks, and the call's epoch
     const int64_t base_a = (int64_t)b * BPB + (int64_t)warp * (C * 32);
@@ -519,7 +538,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                         if (e < N) c += __ldg(tq + src) + (has_rep ? 0 : __ldg(tq + N + src));
                         else c += __ldg(tq + N + src);
                     }
-                if (b < nblk - 1) st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (uint32_t)c);
+                if (b < nblk - 1) st_relaxed_u32(aggw + (int64_t)e * wstride + b, WORD_READY | (uint32_t)c);
             }
             tc_agg[j] = c;
         }
@@ -545,20 +564,13 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                 if (r >= 0 && ((a / K) & 1)) slot = r;
                 if (slot >= n_slots) { bad = 1; slot = -1; }
             }
-            if (slot_out != nullptr) slot_out[a] = slot;
         }
         rank_r[j] = warp_slot_rank(slot, nbits, my, lane);
         slot_r[j] = slot;
     }
     if (__any_sync(FULL, bad) && lane == 0) atomicOr(&s_err, 2);
     __syncthreads();
-    const int blk_err = s_err;
-    if (multi && blk_err != 0 && tid == 0) {
-        // rare path: the error bit is visible before this block's counts are
-        atomicOr(&ctl->err, blk_err);
-        __threadfence();
-    }
-    __syncthreads();
+    const int blk_err = s_err;  // the published counts carry it (WORD_BAD) to later blocks
 
     // 2. per-slot exclusive prefix over warps; the block's counts, published
     int my_agg[LS_SLOTS_PER_THREAD];
@@ -578,39 +590,56 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
             if (pre_published) {
                 if (tc_agg[j] != run) atomicOr(&s_err, 2);  // the tile histograms do not match the indices
             } else if (multi && b < nblk - 1) {
-                st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (uint32_t)run);
+                st_relaxed_u32(aggw + (int64_t)e * wstride + b, WORD_READY | (blk_err ? WORD_BAD : 0u) | (uint32_t)run);
             }
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: 32 independent loads at a time
-    constexpr int PB = 32;
+    // 3. counts of all earlier blocks, per slot: the slot's row of count
+    //    words, 16-byte vectors, up to 16 vectors (64 blocks) in flight
+    constexpr int PV = 16;
     int excl[LS_SLOTS_PER_THREAD];
-    bool timed_out = false;
+    bool timed_out = false, pred_bad = false;
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
         excl[j] = 0;
         const int e = tid + j * LS_THREADS;
         if (e >= n_slots || b == 0) continue;
+        const uint32_t* row = aggw + (int64_t)e * wstride;
+        const int nv = (b + 3) >> 2;  // vectors holding blocks 0 .. b-1
         uint64_t t0 = 0;
-        for (int q0 = 0; q0 < b; q0 += PB) {
-            uint32_t v[PB];
+        for (int v0 = 0; v0 < nv; v0 += PV) {
+            uint4 v[PV];
 #pragma unroll
-            for (int u = 0; u < PB; ++u)
-                v[u] = q0 + u < b ? ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e) : WORD_READY;
+            for (int u = 0; u < PV; ++u)
+                v[u] = v0 + u < nv ? ld_relaxed_v4(row + 4 * (v0 + u)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int u = 0; u < PB; ++u) {
-                // bounded re-poll of a word this call's block q0+u has not published yet
-                while (!(v[u] & WORD_READY) && !timed_out) {
+            for (int u = 0; u < PV; ++u) {
+                if (v0 + u >= nv) continue;
+                const int q0 = 4 * (v0 + u);  // blocks q0 .. q0+3; those >= b are not predecessors
+                auto ready = [&](const uint4& w) {
+                    return ((w.x & WORD_READY) || q0 >= b) && ((w.y & WORD_READY) || q0 + 1 >= b) &&
+                           ((w.z & WORD_READY) || q0 + 2 >= b) && ((w.w & WORD_READY) || q0 + 3 >= b);
+                };
+                // bounded re-poll of a vector whose words are not all published yet
+                while (!ready(v[u]) && !timed_out) {
                     if (t0 == 0) t0 = globaltimer();
                     else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
                     __nanosleep(64);
-                    v[u] = ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e);
+                    v[u] = ld_relaxed_v4(row + 4 * (v0 + u));
                 }
-                excl[j] += (v[u] & WORD_READY) ? (int)(v[u] & ~WORD_READY) : 0;
+                const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (q0 + k < b && (w4[k] & WORD_READY)) {
+                        excl[j] += (int)(w4[k] & WORD_COUNT);
+                        pred_bad |= (w4[k] & WORD_BAD) != 0;
+                    }
+                }
             }
         }
     }
+    if (pred_bad) atomicOr(&s_err, 2);
     if (timed_out) atomicOr(&s_err, 1);
 #pragma unroll
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
@@ -619,30 +648,37 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     }
     __syncthreads();
 
-    // 4. in-expert ranks
+    // 4. in-expert ranks (and the slots, stored here rather than in the
+    //    histogram loop so that no store sits between its chunks)
 #pragma unroll
     for (int j = 0; j < C; ++j) {
         const int64_t a = base_a + j * 32 + lane;
-        if (a < A) rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+        if (a < A) {
+            rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
+            if (slot_out != nullptr) slot_out[a] = slot_r[j];
+        }
     }
 
     // 5. the last block: totals = earlier blocks + its own counts
     if (b == nblk - 1 && counts != nullptr) {
+        // errors: this block's, its predecessors' bad ids (carried in their
+        // counts), and whatever else other blocks have recorded by now (the
+        // workspace status has every one)
+        const int other_err = multi ? ld_volatile(&ctl->err) : 0;  // its latency overlaps the totals
+        __syncthreads();  // ranks read ex and my before wh is reused for the totals
         const int local_err = s_err;
-        if (multi) __threadfence();  // other blocks' error bits, published before their counts, are visible
-        __syncthreads();             // ranks read ex and my before wh is reused for the totals
 #pragma unroll
         for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
             const int e = tid + j * LS_THREADS;
             if (e < n_slots) wh[e] = excl[j] + my_agg[j];
         }
         __syncthreads();
-        finish_totals(wh, true, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T,
-                      multi ? &ctl->err : nullptr, local_err, s_scan, s_red, wh);
+        finish_totals(wh, true, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T, nullptr,
+                      local_err | other_err, s_scan, s_red, wh);
     }
     if (multi) {
         __syncthreads();
-        if (tid == 0 && (s_err & ~blk_err)) atomicOr(&ctl->err, s_err & ~blk_err);  // timeouts, histogram mismatch
+        if (tid == 0 && s_err) atomicOr(&ctl->err, s_err);  // bad ids, timeouts, histogram mismatch
         __syncthreads();
         // the last block to finish clears this call's count words (no block
         // reads them any more) and resets the control words
@@ -654,7 +690,8 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         __syncthreads();
         if (s_last) {
             __threadfence();
-            for (int64_t i = tid; i < (int64_t)(nblk - 1) * n_slots; i += LS_THREADS) aggw[i] = 0u;
+            uint4* w4 = reinterpret_cast<uint4*>(aggw);
+            for (int64_t i = tid; i < (int64_t)n_slots * (wstride / 4); i += LS_THREADS) w4[i] = make_uint4(0, 0, 0, 0);
             if (tid == 0) {
                 ctl->sticky |= ctl->err;
                 ctl->err = 0;

@@ -12,7 +12,6 @@
 // every reduction is a butterfly of shuffles; nothing goes through shared
 // memory.  The order (key desc, index asc) is total, so the result is unique.
 #include <math.h>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "select.cuh"
@@ -215,215 +214,6 @@ cudaError_t launch_capacity_candidates(const float* scores, const float* bias, i
 }
 
 // ---------------------------------------------------------------------------
-// Filtered selection: S = N/32 threads per token, thread j owning experts
-// [32j, 32j+32) (with groups: exactly one group of 32).
-//   1. each thread: keys = fp32(s + b) of its 32 experts and their two
-//      largest (t1 >= t2); with groups, the group score fp32(t1 + t2) (or t1);
-//   2. group ranks by shuffles among the token's S threads; non-kept groups
-//      drop out;
-//   3. theta = the smallest t2 over the candidate threads (2 known keys
-//      each, 2 * candidate threads >= K); if too many keys pass it (a few
-//      groups holding most large keys), the K-th largest of the candidate
-//      threads' four largest keys instead.  Either way at least K candidate
-//      keys are >= theta, so the K best keys are all >= theta;
-//   4. keys >= theta (typically about ten per token) are compacted into a
-//      per-token shared-memory list, in expert order (thread-major, then
-//      ascending index);
-//   5. the token's threads rank the survivors in parallel (rank = how many
-//      survivors beat it in the (key desc, index asc) order) and place the K
-//      best at their ranks; the leader writes weights in k order.  A token
-//      with more survivors than its list holds (32, or 16 for N = 64) takes
-//      a slow path: its leader re-reads the whole row.
-// The result equals the plain definition: the set of keys >= theta contains
-// the top K of the candidates, and the list's order is (key desc, index asc).
-// ---------------------------------------------------------------------------
-constexpr int SEL_THREADS = 256;
-
-template <int S>
-__global__ void __launch_bounds__(SEL_THREADS, 3) route_select_kernel(
-    const float* __restrict__ scores, const float* __restrict__ bias, int T, int K, int grouped,
-    int topk_groups, int group_topn, int renorm, float route_scale, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w) {
-    constexpr int N = 32 * S;
-    constexpr int TPB = SEL_THREADS / S;       // tokens per block
-    constexpr int SEL_CAP = S >= 4 ? 32 : 16;  // survivors kept per token in shared memory
-    // bias transposed, bias_t[i * S + j] = bias[32 * j + i]: the S threads of a
-    // token read consecutive words for the same i (no bank conflicts)
-    __shared__ float bias_t[N];
-    // lists padded by one word: the tokens of a warp start in different banks
-    __shared__ float c_key[TPB][SEL_CAP + 1], c_s[TPB][SEL_CAP + 1];
-    __shared__ int c_idx[TPB][SEL_CAP + 1];
-    __shared__ float o_s[TPB][8];
-    __shared__ int o_i[TPB][8];
-    for (int e = threadIdx.x; e < N; e += blockDim.x) bias_t[(e & 31) * S + (e >> 5)] = bias != nullptr ? bias[e] : 0.f;
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31;
-    const int j = threadIdx.x % S;                 // which 32 experts
-    const int lt = threadIdx.x / S;                // token slot in the block
-    const int seg = lane - (lane % S);             // first lane of this token's segment
-    const float* bj = bias_t + j;  // bias of expert 32 j + i at bj[i * S]
-
-    for (int64_t t0 = (int64_t)blockIdx.x * TPB; t0 < T; t0 += (int64_t)gridDim.x * TPB) {
-        const int64_t t = t0 + lt;
-        const bool live = t < T;
-        // the keys stay in registers; the few survivors' unbiased scores are
-        // re-read (L1 hits) when they are compacted
-        const float* my_row = scores + t * N + 32 * j;
-        float kv[32];
-        if (live) {
-            const float4* src = reinterpret_cast<const float4*>(my_row);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 f = __ldg(src + q);
-                kv[4 * q] = __fadd_rn(f.x, bj[(4 * q) * S]);
-                kv[4 * q + 1] = __fadd_rn(f.y, bj[(4 * q + 1) * S]);
-                kv[4 * q + 2] = __fadd_rn(f.z, bj[(4 * q + 2) * S]);
-                kv[4 * q + 3] = __fadd_rn(f.w, bj[(4 * q + 3) * S]);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) kv[i] = bj[i * S];
-        }
-        // 1. two largest keys of my 32 experts
-        float t1 = -INFINITY, t2 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float key = kv[i];
-            t2 = key > t1 ? t1 : (key > t2 ? key : t2);
-            t1 = key > t1 ? key : t1;
-        }
-        // 2. group ranks among the token's S threads
-        bool cand = true;
-        if (grouped) {
-            const float gs = group_topn == 1 ? t1 : __fadd_rn(t1, t2);
-            int rank = 0;
-#pragma unroll
-            for (int h = 0; h < S; ++h) {
-                const float gh = __shfl_sync(FULL, gs, seg + h);
-                rank += (h != j && beats(gh, h, gs, j)) ? 1 : 0;
-            }
-            cand = rank < topk_groups;
-        }
-        // 3. theta, cheaply: the smallest t2 over the candidate threads (2 known
-        //    keys each).  Tokens whose survivors would not fit the list (a few
-        //    groups holding most large keys) tighten it to the K-th largest of
-        //    the candidate threads' four largest keys, ranked by shuffles.
-        float th = cand ? t2 : INFINITY;
-#pragma unroll
-        for (int o = 1; o < S; o <<= 1) th = fminf(th, __shfl_xor_sync(FULL, th, o));
-        unsigned m = 0;
-        if (cand) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) m |= (kv[i] >= th ? 1u : 0u) << i;
-        }
-        int total = __popc(m);
-#pragma unroll
-        for (int o = 1; o < S; o <<= 1) total += __shfl_xor_sync(FULL, total, o);
-        if (__any_sync(FULL, total > SEL_CAP && live)) {
-            const bool tighten = total > SEL_CAP;
-            float q4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (cand) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float key = kv[i];
-                    const bool g1 = key > q4[0], g2 = key > q4[1], g3 = key > q4[2], g4 = key > q4[3];
-                    q4[3] = g3 ? q4[2] : (g4 ? key : q4[3]);
-                    q4[2] = g2 ? q4[1] : (g3 ? key : q4[2]);
-                    q4[1] = g1 ? q4[0] : (g2 ? key : q4[1]);
-                    q4[0] = g1 ? key : q4[0];
-                }
-            }
-            int rk[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int h = 0; h < S; ++h) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float u = __shfl_sync(FULL, q4[q], seg + h);
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        rk[r] += (u > q4[r] || (u == q4[r] && (h * 4 + q) < (j * 4 + r))) ? 1 : 0;
-                }
-            }
-            float th2 = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-                if (rk[r] == K - 1) th2 = q4[r];
-#pragma unroll
-            for (int o = 1; o < S; o <<= 1) th2 = fmaxf(th2, __shfl_xor_sync(FULL, th2, o));
-            if (tighten) {
-                th = th2;
-                m = 0;
-                if (cand) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) m |= (kv[i] >= th ? 1u : 0u) << i;
-                }
-            }
-            total = __popc(m);
-#pragma unroll
-            for (int o = 1; o < S; o <<= 1) total += __shfl_xor_sync(FULL, total, o);
-        }
-        // 4. survivors: offsets within the token (thread order), compaction
-        const int cnt = __popc(m);
-        int off = cnt;
-#pragma unroll
-        for (int o = 1; o < S; o <<= 1) {
-            const int y = __shfl_up_sync(FULL, off, o, S);
-            if (j >= o) off += y;
-        }
-        off -= cnt;
-        if (total <= SEL_CAP) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if ((m >> i) & 1u) {
-                    c_key[lt][off] = kv[i];
-                    c_s[lt][off] = __ldg(my_row + i);
-                    c_idx[lt][off] = 32 * j + i;
-                    ++off;
-                }
-            }
-        }
-        const unsigned keepbits = (__ballot_sync(FULL, cand) >> seg) & ((1u << S) - 1u);
-        __syncwarp();
-        if (total <= SEL_CAP) {
-            // 5. each of the token's threads ranks a share of the survivors; a
-            //    survivor beaten by fewer than K others is placed at its rank
-            for (int c = j; c < total; c += S) {
-                const float kc = c_key[lt][c];
-                const int ic = c_idx[lt][c];
-                int rank = 0;
-                for (int c2 = 0; c2 < total; ++c2) rank += beats(c_key[lt][c2], c_idx[lt][c2], kc, ic) ? 1 : 0;
-                if (rank < K) { o_i[lt][rank] = ic; o_s[lt][rank] = c_s[lt][c]; }
-            }
-            __syncwarp();
-            if (live) {
-                // every thread forms the same k-ordered sum; thread k writes slot k
-                float ssum = o_s[lt][0];
-                for (int k = 1; k < K; ++k) ssum = __fadd_rn(ssum, o_s[lt][k]);
-                for (int k = j; k < K; k += S) {
-                    const float wv = renorm ? __fdiv_rn(o_s[lt][k], ssum) : o_s[lt][k];
-                    topk_idx[t * K + k] = o_i[lt][k];
-                    topk_w[t * K + k] = __fmul_rn(wv, route_scale);
-                }
-            }
-        } else if (j == 0 && live) {
-            // slow path: the leader re-reads the whole row
-            Top8 top;
-            top.init();
-            const float* row = scores + t * N;
-            for (int e = 0; e < N; ++e) {
-                if (!((keepbits >> (e >> 5)) & 1u)) continue;
-                const float sv = row[e];
-                const float key = __fadd_rn(sv, bias_t[(e & 31) * S + (e >> 5)]);
-                if (key >= th) top.offer(key, e, sv);
-            }
-            top.write(K, renorm, route_scale, topk_idx + t * K, topk_w + t * K);
-        }
-        __syncwarp();
-    }
-}
-
-// ---------------------------------------------------------------------------
 // Warp-per-token selection.  Lane l owns experts [l*EPL, l*EPL + EPL)
 // (EPL = N/32), so an expert group of 32 spans G = 32/EPL consecutive lanes;
 // the lane's bias values live in registers for the whole kernel.
@@ -597,16 +387,6 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
     }
 }
 
-// The filtered kernel covers N in {64, 128, 256}, K <= 8, and either one
-// group or groups of exactly 32 experts with a group score of the top one or
-// two keys, when the candidate threads hold at least K known keys (2 each).
-static bool select_fast_ok(int N, int K, int n_groups, int topk_groups, int group_topn) {
-    if (!(N == 64 || N == 128 || N == 256) || K > 8) return false;
-    const int S = N / 32;
-    if (n_groups == 1) return 2 * S >= K;
-    return N / n_groups == 32 && group_topn >= 1 && group_topn <= 2 && 2 * topk_groups >= K;
-}
-
 // Elements per lane for N experts; 0 if unsupported.
 int route_epl(int N) {
     if (N <= 32) return 1;
@@ -628,9 +408,7 @@ static bool select_warp_ok(int N, int K, int n_groups, int group_topn) {
 cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int N, int K,
                               int n_groups, int topk_groups, int group_topn, int renorm,
                               float route_scale, int32_t* idx, float* w, cudaStream_t st) {
-    const char* env = getenv("MOE_SELECT_KERNEL");  // "filtered": the thread-per-group kernel (measurement)
-    const bool filtered = env != nullptr && env[0] == 'f';
-    if (!filtered && select_warp_ok(N, K, n_groups, group_topn)) {
+    if (select_warp_ok(N, K, n_groups, group_topn)) {
         // one wave of resident blocks (three per SM at this kernel's registers); each warp
         // walks its tokens with the next row's load in flight
         long long blocks = ((long long)T + SW_THREADS / 32 - 1) / (SW_THREADS / 32);
@@ -648,24 +426,6 @@ cudaError_t launch_route_topk(const float* scores, const float* bias, int T, int
             default: MOE_SELW(16); break;
         }
 #undef MOE_SELW
-        moe_host::note_launch();
-        return cudaGetLastError();
-    }
-    if (select_fast_ok(N, K, n_groups, topk_groups, group_topn)) {
-        const int S = N / 32;
-        long long blocks = ((long long)T * S + SEL_THREADS - 1) / SEL_THREADS;
-        const long long cap = (long long)moe_host::sm_count() * 16;
-        if (blocks > cap) blocks = cap;
-        if (blocks < 1) blocks = 1;
-        const int grouped = n_groups > 1 ? 1 : 0;
-        switch (S) {
-            case 2: route_select_kernel<2><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
-                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
-            case 4: route_select_kernel<4><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
-                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
-            default: route_select_kernel<8><<<(unsigned)blocks, SEL_THREADS, 0, st>>>(
-                        scores, bias, T, K, grouped, topk_groups, group_topn, renorm, route_scale, idx, w); break;
-        }
         moe_host::note_launch();
         return cudaGetLastError();
     }

@@ -33,18 +33,31 @@ from . import moe
 PIPELINED_GATE_CTAS = 64
 
 
+def fused_routing_supported(wl, x) -> bool:
+    """Whether moe_route_tiles takes this workload: bf16 tokens on the
+    tensor-core gate (64, 128 or 256 experts), K <= 8, and one group or
+    sigmoid groups of 32 experts scored by their top one or two keys."""
+    xs = x[0] if isinstance(x, (list, tuple)) else x
+    if xs.dtype != torch.bfloat16 or wl.N not in (64, 128, 256) or wl.K > 8:
+        return False
+    return wl.n_groups == 1 or (wl.fn == moe.MOE_SIGMOID and wl.N // wl.n_groups == 32 and wl.group_topn <= 2)
+
+
 class RoutingStep:
     """x: the token batch [T, d], or a list of batches that step() cycles
     through when it is given none (consecutive batches then live in
     different buffers, as in a stream of distinct batches)."""
 
     def __init__(self, wl, x, w_gate, bias, logit_offset, device, world: int = 1, pipelined: bool = True,
-                 gate_max_ctas: int | None = None, bias_rate: float = 0.001, fused: bool = False):
+                 gate_max_ctas: int | None = None, bias_rate: float = 0.001, fused: bool | None = None):
         T, d, N, K = wl.T, wl.d, wl.N, wl.K
         self.wl, self.dev, self.world, self.pipelined, self.u = wl, device, world, pipelined, bias_rate
         # fused: the selection and a per-tile histogram in the gate's epilogue
         # (moe_route_tiles, no scores in memory), statistics from those
-        # histograms (moe_load_stats_tiles)
+        # histograms (moe_load_stats_tiles).  Default: wherever the epilogue
+        # can select (the shapes moe_route_tiles accepts).
+        if fused is None:
+            fused = fused_routing_supported(wl, x)
         self.fused = fused
         self.batches = list(x) if isinstance(x, (list, tuple)) else [x]
         x = self.batches[0]
