@@ -874,8 +874,9 @@ def run_report(oracle_seconds: float = 4.0):
         return a.elapsed_time(b) / n * 1e3
 
     P("## 3. Routed tokens/s per workload: the GPU pipeline beside the oracle\n")
-    P(f"GPU: route (gate + selection) -> load statistics (+ replica plan and the slot remap for the prefill "
-      f"workload) -> bias step (workloads with a bias) -> dispatch (+ FP8 copy for the softmax-dispatch "
+    P(f"GPU: route (gate + selection; '(fused)': selection and tile histograms in the gate's epilogue, "
+      f"moe_route_tiles + moe_load_stats_tiles) -> load statistics (+ replica plan and the slot remap for the "
+      f"prefill workload) -> bias step (workloads with a bias) -> dispatch (+ FP8 copy for the softmax-dispatch "
       f"workload), one stream, 10 pipelines captured in a CUDA graph and replayed under CUDA events.  Roofline = "
       f"sum over the stages of max(bytes / {hbm:.1f} GB/s, gate flops / {tf_burst:.1f} TFLOP/s) ({peak_kind} "
       f"peaks).  Oracle: the same stage set in plain C (fp64), on a bounded sample of each workload's tokens, on "
@@ -908,32 +909,47 @@ def run_report(oracle_seconds: float = 4.0):
         sc = torch.empty(A, d // 128, device=dev) if wl.fp8 else None
         pos = torch.empty(T, K, dtype=torch.int32, device=dev)
 
+        from expert_load_balancing_tcgen05_b200.step import fused_routing_supported
+        fused = fused_routing_supported(wl, x)
+        tiles = torch.empty(moe.tile_counts_shape(T, N), dtype=torch.int32, device=dev) if fused else None
+
+        def stats_call(rep, ns, cnt, offs):
+            if fused:
+                moe.moe_load_stats_tiles(idx, T, K, N, tiles, rep, ns, slot, cnt, offs, rank, stats, ws)
+            else:
+                moe.moe_load_stats(idx, T, K, N, rep, ns, slot, cnt, offs, rank, None, wl.fn, stats, ws)
+
         def pipeline():
-            moe.moe_route(cfg, x, Wg, off, b2, scores, idx, w, ws)
+            if fused:
+                moe.moe_route_tiles(cfg, x, Wg, off, b2, idx, w, tiles, ws)
+            else:
+                moe.moe_route(cfg, x, Wg, off, b2, scores, idx, w, ws)
             if rs is not None:
-                moe.moe_load_stats(idx, T, K, N, None, N, slot, counts[:N], offsets[:N + 1], rank, None, wl.fn,
-                                   stats, ws)
+                stats_call(None, N, counts[:N], offsets[:N + 1])
                 moe.moe_replica_plan(counts[:N], N, wl.n_replicas, rs)
-            moe.moe_load_stats(idx, T, K, N, rs, wl.n_slots, slot, counts, offsets, rank, None, wl.fn, stats, ws)
+            stats_call(rs, wl.n_slots, counts, offsets)
             if b2 is not None:
                 moe.moe_bias_update(counts[:N], N, A, 0.001, 0, b2)
             moe.moe_dispatch(x, T, d, K, slot, offsets, rank, rows, q, sc, pos, None)
 
         us = t_us(pipeline)
-        nbytes = (T * d * es + N * d * es + T * N * 4 + A * 8) + (T * N * 4 + A * 8) + A * 12 + \
-            (T * d * es + A * d * es + A * 12) + ((A * d + A * d // 32) if wl.fp8 else 0)
+        # route bytes: the fused path never writes or re-reads the scores
+        route_b = (T * d * es + N * d * es + A * 8 + tiles.numel() * 4) if fused else \
+            (T * d * es + N * d * es + T * N * 4 + A * 8) + (T * N * 4 + A * 8)
+        nbytes = route_b + A * 12 + (T * d * es + A * d * es + A * 12) + ((A * d + A * d // 32) if wl.fp8 else 0)
         # serial roofline: the gate at the slower of its HBM and tensor bounds, the rest at HBM speed
-        gate_b = T * d * es + N * d * es + T * N * 4
+        gate_b = T * d * es + N * d * es + (A * 8 if fused else T * N * 4)
         roof = (max(gate_b / (hbm * 1e9), 2 * T * d * N / (tf_burst * 1e12)) + (nbytes - gate_b) / (hbm * 1e9)) * 1e6
         gpu_tps = T / (us / 1e6)
-        del inp, x, Wg, scores, idx, w, ws, slot, rank, rows, q, sc, pos
+        del inp, x, Wg, scores, idx, w, ws, slot, rank, rows, q, sc, pos, tiles
         torch.cuda.empty_cache()
         o_tps, n, dt, used = _oracle_rate(wl, oracle_seconds)
         one = ""
         if name in ("tiny_softmax", "v3_router"):
             o1, n1, dt1, _ = _oracle_rate(wl, oracle_seconds, threads=1)
             one = f"{o1:,.0f} ({n1}, {dt1:.1f} s)"
-        P(f"| {name} | T={T} d={d} N={N} K={K} | {us:.1f} | {gpu_tps:,.0f} | {nbytes / (us / 1e6) / 1e9:,.0f} | "
+        P(f"| {name}{' (fused)' if fused else ''} | T={T} d={d} N={N} K={K} | {us:.1f} | {gpu_tps:,.0f} | "
+          f"{nbytes / (us / 1e6) / 1e9:,.0f} | "
           f"{roof / us:.2f} | {o_tps:,.0f} ({used}) | {n}, {dt:.1f} s | {one or '-'} | "
           f"{gpu_tps / o_tps:,.0f} |")
     P("")

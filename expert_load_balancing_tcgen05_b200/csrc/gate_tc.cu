@@ -145,6 +145,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 8 columns: the fused epilogue's selection loops walk a chunk in these
+// pieces so that their (rolled) bodies stay small enough for the instruction
+// cache -- each offer into the sorted list unrolls to dozens of instructions
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 template <int BN>
 struct Cfg {
     static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
@@ -176,6 +189,11 @@ struct Epi {
 __device__ __forceinline__ void store32(float* dst, const float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+}
+
+__device__ __forceinline__ void store8(float* dst, const float (&v)[8]) {
+    *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
 // Named barrier over the epilogue warps only.
@@ -211,7 +229,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
     if (p.fn == MOE_SIGMOID) {
         if (FUSED && p.n_groups > 1) {
             // one expert group per 32-column chunk: group score = sum of its top-n keys
-#pragma unroll
+#pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
                 tmem_ld32(taddr + 32 * c, v);
@@ -240,14 +258,33 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
-                tmem_ld32(taddr + 32 * c, v);  // warp-collective: every lane loads every chunk
-                if ((keep >> c) & 1u) {
+                const bool kc = (keep >> c) & 1u;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float v8[8];
+                    tmem_ld8(taddr + 32 * c + 8 * q, v8);  // warp-collective: every lane loads every piece
+                    if (kc) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float sv = sigmoid_f(v[i] + off_s[32 * c + i]);
-                        top.offer(__fadd_rn(sv, bias_s[32 * c + i]), 32 * c + i, sv);
+                        for (int i = 0; i < 8; ++i) {
+                            const int col = 32 * c + 8 * q + i;
+                            const float sv = sigmoid_f(v8[i] + off_s[col]);
+                            top.offer(__fadd_rn(sv, bias_s[col]), col, sv);
+                        }
                     }
                 }
+            }
+        } else if constexpr (FUSED) {
+#pragma unroll 1
+            for (int q = 0; q < 4 * NCH; ++q) {
+                const int col0 = 32 * c_lo + 8 * q;
+                float v8[8];
+                tmem_ld8(taddr + col0, v8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    v8[i] = sigmoid_f(v8[i] + off_s[col0 + i]);
+                    top.offer(__fadd_rn(v8[i], bias_s[col0 + i]), col0 + i, v8[i]);
+                }
+                if (srow) store8(srow + col0, v8);
             }
         } else {
 #pragma unroll 1
@@ -255,10 +292,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 const int c = c_lo + cc;
                 tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
-                    if constexpr (FUSED) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
-                }
+                for (int i = 0; i < 32; ++i) v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
                 if (srow) store32(srow + 32 * c, v);
             }
         }
@@ -286,16 +320,28 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
         x.red[(h * 2 + 1) * BM + row] = sum;
         epi_sync();
         const float inv = 1.f / (x.red[1 * BM + row] + x.red[3 * BM + row]);
+        if constexpr (FUSED) {
 #pragma unroll 1
-        for (int cc = 0; cc < NCH; ++cc) {
-            const int c = c_lo + cc;
-            tmem_ld32(taddr + 32 * c, v);
+            for (int q = 0; q < 4 * NCH; ++q) {
+                const int col0 = 32 * c_lo + 8 * q;
+                float v8[8];
+                tmem_ld8(taddr + col0, v8);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
-                if constexpr (FUSED) top.offer(__fadd_rn(v[i], bias_s[32 * c + i]), 32 * c + i, v[i]);
+                for (int i = 0; i < 8; ++i) {
+                    v8[i] = expf(v8[i] + off_s[col0 + i] - m) * inv;
+                    top.offer(__fadd_rn(v8[i], bias_s[col0 + i]), col0 + i, v8[i]);
+                }
+                if (srow) store8(srow + col0, v8);
             }
-            if (srow) store32(srow + 32 * c, v);
+        } else {
+#pragma unroll 1
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int c = c_lo + cc;
+                tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
+                if (srow) store32(srow + 32 * c, v);
+            }
         }
     }
     if constexpr (!FUSED) return;

@@ -484,10 +484,16 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     int n_slots, int32_t* __restrict__ slot_out, int32_t* __restrict__ rank_out, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, moe_stats* stats, const double* __restrict__ hs_partial, int hs_blocks,
     int64_t T, ScanCtl* ctl, uint32_t* aggw, int nblk, int block_base, const int32_t* __restrict__ tile_counts) {
+    // Each SM runs one block of this kernel once, so its instructions are
+    // fetched cold: the loops stay rolled (their bodies then run from the
+    // instruction cache) and the block's ids, slots and ranks live in shared
+    // memory rather than in fully unrolled registers.
     constexpr int BPB = LS_WARPS * C * 32;
     extern __shared__ int32_t sm_dyn[];
     int32_t* wh = sm_dyn;                       // [LS_WARPS][n_slots]
     int32_t* ex = sm_dyn + LS_WARPS * n_slots;  // [n_slots] earlier-block counts
+    int32_t* s_slot = ex + n_slots;             // [BPB] this block's expert ids, then slots
+    int32_t* s_rank = s_slot + BPB;             // [BPB] in-warp ranks
     __shared__ int s_err;
     __shared__ int s_scan[33];
     __shared__ double s_red[32];
@@ -495,15 +501,11 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     const int b = block_base + (int)blockIdx.x;  // block_base > 0 only in the bounded-wait self-test
     const bool multi = nblk > 1;
     const int wstride = word_stride(nblk);  // count words: aggw[slot * wstride + block]
+    const int64_t a0 = (int64_t)b * BPB;
 
-    // the loads first: expert ids of this warp's chunks, and the call's epoch
-    const int64_t base_a = (int64_t)b * BPB + (int64_t)warp * (C * 32);
-    int slot_r[C], rank_r[C];
-#pragma unroll
-    for (int j = 0; j < C; ++j) {
-        const int64_t a = base_a + j * 32 + lane;
-        slot_r[j] = a < A ? __ldg(idx + a) : -1;
-    }
+    // the block's expert ids (eight independent loads per thread in flight)
+#pragma unroll 8
+    for (int v = tid; v < BPB; v += LS_THREADS) s_slot[v] = a0 + v < A ? __ldg(idx + a0 + v) : -1;
     if (tid == 0) s_err = 0;
     for (int i = tid; i < LS_WARPS * n_slots; i += LS_THREADS) wh[i] = 0;
     // the gate epilogue's per-tile histograms (tiles of 128 tokens, aligned to
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                 if (r >= N && r < n_slots) ex[r - N] = e;
             }
         __syncthreads();
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
             const int e = tid + j * LS_THREADS;
             int c = 0;
@@ -545,14 +547,15 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     }
     __syncthreads();
 
-    // 1. slots, warp histograms, in-warp stable ranks
+    // 1. slots, warp histograms, in-warp stable ranks (one chunk of 32 per step)
     int32_t* my = wh + warp * n_slots;
     const int nbits = n_slots > 1 ? 32 - __clz(n_slots - 1) : 0;
     int bad = 0;
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < C; ++j) {
-        const int64_t a = base_a + j * 32 + lane;
-        int slot = slot_r[j];
+        const int li = warp * (C * 32) + j * 32 + lane;
+        const int64_t a = a0 + li;
+        int slot = s_slot[li];
         if (a < A) {
             if (slot < 0) {
                 slot = -1;  // dropped by the capacity limit: no slot, rank -1
@@ -565,8 +568,8 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                 if (slot >= n_slots) { bad = 1; slot = -1; }
             }
         }
-        rank_r[j] = warp_slot_rank(slot, nbits, my, lane);
-        slot_r[j] = slot;
+        s_rank[li] = warp_slot_rank(slot, nbits, my, lane);
+        s_slot[li] = slot;
     }
     if (__any_sync(FULL, bad) && lane == 0) atomicOr(&s_err, 2);
     __syncthreads();
@@ -595,49 +598,44 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: the slot's row of count
-    //    words, 16-byte vectors, up to 16 vectors (64 blocks) in flight
-    constexpr int PV = 16;
+    // 3. counts of all earlier blocks, per slot: its row of count words,
+    //    eight at a time (two 16-byte loads)
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false, pred_bad = false;
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < LS_SLOTS_PER_THREAD; ++j) {
         excl[j] = 0;
         const int e = tid + j * LS_THREADS;
         if (e >= n_slots || b == 0) continue;
         const uint32_t* row = aggw + (int64_t)e * wstride;
-        const int nv = (b + 3) >> 2;  // vectors holding blocks 0 .. b-1
         uint64_t t0 = 0;
-        for (int v0 = 0; v0 < nv; v0 += PV) {
-            uint4 v[PV];
+        int acc = 0;
+#pragma unroll 1
+        for (int q0 = 0; q0 < b; q0 += 8) {
+            uint32_t w8[8];
+            {
+                const uint4 lo = ld_relaxed_v4(row + q0);
+                const uint4 hi = q0 + 4 < wstride ? ld_relaxed_v4(row + q0 + 4) : make_uint4(0, 0, 0, 0);
+                w8[0] = lo.x; w8[1] = lo.y; w8[2] = lo.z; w8[3] = lo.w;
+                w8[4] = hi.x; w8[5] = hi.y; w8[6] = hi.z; w8[7] = hi.w;
+            }
 #pragma unroll
-            for (int u = 0; u < PV; ++u)
-                v[u] = v0 + u < nv ? ld_relaxed_v4(row + 4 * (v0 + u)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int u = 0; u < PV; ++u) {
-                if (v0 + u >= nv) continue;
-                const int q0 = 4 * (v0 + u);  // blocks q0 .. q0+3; those >= b are not predecessors
-                auto ready = [&](const uint4& w) {
-                    return ((w.x & WORD_READY) || q0 >= b) && ((w.y & WORD_READY) || q0 + 1 >= b) &&
-                           ((w.z & WORD_READY) || q0 + 2 >= b) && ((w.w & WORD_READY) || q0 + 3 >= b);
-                };
-                // bounded re-poll of a vector whose words are not all published yet
-                while (!ready(v[u]) && !timed_out) {
+            for (int u = 0; u < 8; ++u) {
+                if (q0 + u >= b) break;
+                // bounded re-poll of a word block q0+u has not published yet
+                while (!(w8[u] & WORD_READY) && !timed_out) {
                     if (t0 == 0) t0 = globaltimer();
                     else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
                     __nanosleep(64);
-                    v[u] = ld_relaxed_v4(row + 4 * (v0 + u));
+                    w8[u] = ld_relaxed_u32(row + q0 + u);
                 }
-                const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    if (q0 + k < b && (w4[k] & WORD_READY)) {
-                        excl[j] += (int)(w4[k] & WORD_COUNT);
-                        pred_bad |= (w4[k] & WORD_BAD) != 0;
-                    }
+                if (w8[u] & WORD_READY) {
+                    acc += (int)(w8[u] & WORD_COUNT);
+                    pred_bad |= (w8[u] & WORD_BAD) != 0;
                 }
             }
         }
+        excl[j] = acc;
     }
     if (pred_bad) atomicOr(&s_err, 2);
     if (timed_out) atomicOr(&s_err, 1);
@@ -648,14 +646,15 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     }
     __syncthreads();
 
-    // 4. in-expert ranks (and the slots, stored here rather than in the
-    //    histogram loop so that no store sits between its chunks)
-#pragma unroll
+    // 4. in-expert ranks, and the slots
+#pragma unroll 4
     for (int j = 0; j < C; ++j) {
-        const int64_t a = base_a + j * 32 + lane;
+        const int li = warp * (C * 32) + j * 32 + lane;
+        const int64_t a = a0 + li;
         if (a < A) {
-            rank_out[a] = slot_r[j] >= 0 ? ex[slot_r[j]] + my[slot_r[j]] + rank_r[j] : -1;
-            if (slot_out != nullptr) slot_out[a] = slot_r[j];
+            const int sl = s_slot[li];
+            rank_out[a] = sl >= 0 ? ex[sl] + my[sl] + s_rank[li] : -1;
+            if (slot_out != nullptr) slot_out[a] = sl;
         }
     }
 
@@ -845,14 +844,15 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
         uint32_t* aggw = reinterpret_cast<uint32_t*>(agg);  // one ready-flagged count word per (block, slot)
         auto kern = chunks == 8 ? load_stats_v2_kernel<8> : (chunks == 16 ? load_stats_v2_kernel<16>
                                                                           : load_stats_v2_kernel<32>);
-        if (lsm > 48 * 1024) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm);
+        const size_t lsm2 = lsm + sizeof(int32_t) * 2 * (size_t)LS_THREADS * chunks;  // + ids/slots and ranks
+        if (lsm2 > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm2);
             if (e != cudaSuccess) return e;
         }
         // the tile histograms serve when a block is a whole number of 128-token tiles
         const int bpb = LS_THREADS * chunks;
         const bool tiles_ok = tile_counts != nullptr && bpb % K == 0 && (bpb / K) % 128 == 0;
-        kern<<<nb, LS_THREADS, lsm, st>>>(idx, A, K, N, replica_slot, n_slots, slot_idx, rank, counts, offsets, stats,
+        kern<<<nb, LS_THREADS, lsm2, st>>>(idx, A, K, N, replica_slot, n_slots, slot_idx, rank, counts, offsets, stats,
                                           part, HS_BLOCKS, T, ctl, aggw, nb, 0, tiles_ok ? tile_counts : nullptr);
         moe_host::note_launch();
         return cudaGetLastError();
@@ -885,7 +885,7 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
         // cleared by every call's last block)
         cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
         if (e != cudaSuccess) return e;
-        const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8;
+        const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8 + (probe == 1 ? sizeof(int32_t) * 2 * LS_BLOCK : 0);
         if (probe == 0)
             load_stats_kernel<<<1, LS_THREADS, smem, st>>>(
                 nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,

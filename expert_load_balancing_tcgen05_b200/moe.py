@@ -15,7 +15,8 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoeroute.so")
+# MOEROUTE_LIB names another build of the library (for side-by-side timing)
+LIB_PATH = os.environ.get("MOEROUTE_LIB") or os.path.join(_HERE, "libmoeroute.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
