@@ -19,18 +19,21 @@ constexpr unsigned FULL = 0xffffffffu;
 //   header   256 B   gate error word (moe_route)
 //   ctl       64 B   per-call control of the load-statistics pass: tile
 //                    ticket, finished-block counter, error bits
-//   flags   4*nblk   look-back status per block: bit 31 | call epoch << 2 | state
-//                    (state 1 aggregate, 2 prefix); a word without this
-//                    call's tag -- zero, an older call's flag, or a count of
-//                    another layout (counts never have bit 31) -- means "none"
-//   agg     nblk x n_slots int32   per-block slot counts
+//   flags   4*nblk   look-back status per block (look-back kernel): bit 31 |
+//                    call epoch << 2 | state (state 1 aggregate, 2 prefix);
+//                    a word without this call's tag means "none"
+//   agg     nblk x n_slots int32   per-block slot counts (look-back kernel), or
+//                    the chain-free kernel's count words: bit 31 (ready) |
+//                    bit 30 (bad id seen) | count, laid out per slot
 //   pre     nblk x n_slots int32   per-block inclusive prefix over blocks
 //   hs      HS_BLOCKS x N double   score-entropy partial column sums
-// The workspace is zero-filled once by its owner before first use.  Each
-// load-statistics call then leaves ctl ready for the next call (its last
-// block resets the ticket and finished counter and advances the epoch after
-// every other block is done); flags need no reset because they carry the
-// epoch; the error words are sticky until moe_workspace_status reads them.
+// The layout depends on the problem size, so one call's flags can lie where
+// another call's count words go.  Invariant: no call leaves a flagged word
+// behind -- the last block of every load-statistics call, once no block
+// reads them any more, clears that call's look-back flags or count words,
+// resets the ticket and finished counter and advances the epoch.  The
+// workspace is zero-filled once by its owner before first use; the error
+// words are sticky until moe_workspace_status reads them.
 // ---------------------------------------------------------------------------
 struct WsHeader {
     int32_t gate_err;       // bit 0: a barrier wait of the gate GEMM ran out
@@ -59,6 +62,7 @@ constexpr int MAX_SLOTS = 2048;                // smem: 8 warps x 2048 x 4 B = 6
 constexpr int LS_SLOTS_PER_THREAD = MAX_SLOTS / LS_THREADS;
 constexpr int HS_BLOCKS = 256;                 // blocks of the score-entropy pass
 constexpr int V2_MAX_BLOCKS = 320;             // largest grid of the chain-free load-statistics kernel
+constexpr int V2_WAVE = 148;                   // preferred grid: one block per SM of a B200
 constexpr int MAX_N = 1024;                    // experts supported by selection / stats
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -80,7 +84,14 @@ inline WsLayout ws_layout(int64_t T, int32_t K, int32_t N, int32_t n_slots) {
     w.flags = off + sizeof(ScanCtl);
     w.ctl_bytes = sizeof(ScanCtl) + sizeof(uint32_t) * (size_t)w.nblk;
     off += align256(w.ctl_bytes);
-    w.agg = off;         off += align256(sizeof(int32_t) * cells);
+    // the chain-free kernel's count words: n_slots rows of one word per block
+    // of (at least) 1024 assignments, rows rounded to 16-byte vectors; they
+    // share the agg and pre regions
+    const int64_t nblk_fine = (A + 1023) / 1024 < 1 ? 1 : (A + 1023) / 1024;
+    const size_t words = (size_t)n_slots * (size_t)((nblk_fine + 3) & ~int64_t(3));
+    const size_t agg_bytes = sizeof(int32_t) * cells > sizeof(int32_t) * words ? sizeof(int32_t) * cells
+                                                                                : sizeof(int32_t) * words;
+    w.agg = off;         off += align256(agg_bytes);
     w.pre = off;         off += align256(sizeof(int32_t) * cells);
     w.hs_partial = off;  off += align256(sizeof(double) * (size_t)HS_BLOCKS * (size_t)(N > 0 ? N : 1));
     w.total = off;

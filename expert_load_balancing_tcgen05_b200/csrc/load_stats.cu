@@ -220,11 +220,24 @@ __device__ __forceinline__ int warp_slot_rank(int slot, int nbits, int32_t* my, 
 
 // Block end: the last block to finish folds this call's error bits into the
 // sticky word and resets the control words for the next call.
-__device__ __forceinline__ void block_done(ScanCtl* ctl, int64_t nblk) {
+// Every block calls it (whole block, uniformly) as its last step.  The last
+// to finish -- no block reads the look-back flags any more -- clears the
+// call's flags, so that no flagged word outlives its call (the workspace
+// layout depends on the problem size, and another call's count words may
+// land where these flags were), folds the call's error bits into the sticky
+// word and resets the control words.
+__device__ __forceinline__ void block_done(ScanCtl* ctl, uint32_t* flags, int64_t nblk) {
+    __shared__ int s_last_lb;
+    __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1)) {
-            __threadfence();
+        s_last_lb = atomicAdd(&ctl->done, 1u) == (uint32_t)(nblk - 1);
+    }
+    __syncthreads();
+    if (s_last_lb) {
+        __threadfence();
+        for (int64_t i = threadIdx.x; i < nblk; i += blockDim.x) flags[i] = 0u;
+        if (threadIdx.x == 0) {
             ctl->sticky |= ctl->err;
             ctl->err = 0;
             ctl->done = 0;
@@ -264,7 +277,7 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
         // a ticket past the grid: the control words were not reset (two calls
         // overlapped on one workspace).  Write nothing; report it (bit 2).
         if (tid == 0) atomicOr(&ctl->err, 4);
-        block_done(ctl, nblk);
+        block_done(ctl, flags, nblk);
         return;
     }
 
@@ -424,8 +437,7 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
         finish_totals(pre + b * n_slots, false, n_slots, A, counts, offsets, stats, hs_partial, hs_blocks, N, T,
                       &ctl->err, 0, s_scan, s_red, wh);
     }
-    __syncthreads();
-    block_done(ctl, nblk);
+    block_done(ctl, flags, nblk);
 }
 
 // ---------------------------------------------------------------------------
@@ -598,8 +610,9 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: its row of count words,
-    //    eight at a time (two 16-byte loads)
+    // 3. counts of all earlier blocks, per slot: its row of count words, up
+    //    to 64 words (16 vectors) in flight at once
+    constexpr int PV = 16;
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false, pred_bad = false;
 #pragma unroll 1
@@ -610,28 +623,30 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         const uint32_t* row = aggw + (int64_t)e * wstride;
         uint64_t t0 = 0;
         int acc = 0;
+        const int nv = (b + 3) >> 2;  // vectors holding blocks 0 .. b-1
 #pragma unroll 1
-        for (int q0 = 0; q0 < b; q0 += 8) {
-            uint32_t w8[8];
-            {
-                const uint4 lo = ld_relaxed_v4(row + q0);
-                const uint4 hi = q0 + 4 < wstride ? ld_relaxed_v4(row + q0 + 4) : make_uint4(0, 0, 0, 0);
-                w8[0] = lo.x; w8[1] = lo.y; w8[2] = lo.z; w8[3] = lo.w;
-                w8[4] = hi.x; w8[5] = hi.y; w8[6] = hi.z; w8[7] = hi.w;
-            }
+        for (int v0 = 0; v0 < nv; v0 += PV) {
+            uint4 vv[PV];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (q0 + u >= b) break;
-                // bounded re-poll of a word block q0+u has not published yet
-                while (!(w8[u] & WORD_READY) && !timed_out) {
-                    if (t0 == 0) t0 = globaltimer();
-                    else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
-                    __nanosleep(64);
-                    w8[u] = ld_relaxed_u32(row + q0 + u);
-                }
-                if (w8[u] & WORD_READY) {
-                    acc += (int)(w8[u] & WORD_COUNT);
-                    pred_bad |= (w8[u] & WORD_BAD) != 0;
+            for (int u = 0; u < PV; ++u) vv[u] = v0 + u < nv ? ld_relaxed_v4(row + 4 * (v0 + u)) : make_uint4(0, 0, 0, 0);
+#pragma unroll 1
+            for (int u = 0; u < PV && v0 + u < nv; ++u) {
+                const int q0 = 4 * (v0 + u);
+                uint32_t w4[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (q0 + k >= b) break;
+                    // bounded re-poll of a word block q0+k has not published yet
+                    while (!(w4[k] & WORD_READY) && !timed_out) {
+                        if (t0 == 0) t0 = globaltimer();
+                        else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
+                        __nanosleep(64);
+                        w4[k] = ld_relaxed_u32(row + q0 + k);
+                    }
+                    if (w4[k] & WORD_READY) {
+                        acc += (int)(w4[k] & WORD_COUNT);
+                        pred_bad |= (w4[k] & WORD_BAD) != 0;
+                    }
                 }
             }
         }
@@ -837,13 +852,18 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
     const size_t lsm = sizeof(int32_t) * (LS_WARPS + 1) * (size_t)n_slots;
     // problems of up to V2_MAX_BLOCKS blocks of 2048, 4096 or 8192 assignments
     // run without a look-back chain; larger ones use the look-back kernel
-    const int chunks = A <= (int64_t)V2_MAX_BLOCKS / 2 * 2048 ? 8 : (A <= (int64_t)V2_MAX_BLOCKS / 2 * 4096 ? 16 : 32);
+    // the smallest blocks (1024, 2048, 4096 or 8192 assignments) that still
+    // fit one block per SM, or, beyond that, up to V2_MAX_BLOCKS blocks of 8192
+    int chunks = 32;
+    for (int c = 4; c <= 32; c *= 2)
+        if (A <= (int64_t)V2_WAVE * LS_THREADS * c) { chunks = c; break; }
     const int64_t nb2 = (A + (int64_t)LS_THREADS * chunks - 1) / ((int64_t)LS_THREADS * chunks);
     if (nb2 <= V2_MAX_BLOCKS) {
         const int nb = nb2 < 1 ? 1 : (int)nb2;
         uint32_t* aggw = reinterpret_cast<uint32_t*>(agg);  // one ready-flagged count word per (block, slot)
-        auto kern = chunks == 8 ? load_stats_v2_kernel<8> : (chunks == 16 ? load_stats_v2_kernel<16>
-                                                                          : load_stats_v2_kernel<32>);
+        auto kern = chunks == 4 ? load_stats_v2_kernel<4>
+                                : (chunks == 8 ? load_stats_v2_kernel<8>
+                                               : (chunks == 16 ? load_stats_v2_kernel<16> : load_stats_v2_kernel<32>));
         const size_t lsm2 = lsm + sizeof(int32_t) * 2 * (size_t)LS_THREADS * chunks;  // + ids/slots and ranks
         if (lsm2 > 48 * 1024) {
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm2);
@@ -909,6 +929,8 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
         memset(&z, 0, sizeof(z));
         z.epoch = h.epoch + 1;
         if ((e = cudaMemcpyAsync(ctl, &z, sizeof(z), cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
+        // no flag of the probe outlives it (its block published one)
+        if ((e = cudaMemsetAsync(w + L.flags, 0, sizeof(uint32_t) * (size_t)L.nblk, st)) != cudaSuccess) return e;
         if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
     }
     *err_out = bits;
