@@ -23,8 +23,8 @@ constexpr unsigned FULL = 0xffffffffu;
 //                    call epoch << 2 | state (state 1 aggregate, 2 prefix);
 //                    a word without this call's tag means "none"
 //   agg     nblk x n_slots int32   per-block slot counts (look-back kernel), or
-//                    the chain-free kernel's count words: bit 31 (ready) |
-//                    bit 30 (bad id seen) | count, laid out per slot
+//                    the chain-free kernel's count words [block][slot]: bit 31
+//                    (ready) | bit 30 (bad id seen) | count
 //   pre     nblk x n_slots int32   per-block inclusive prefix over blocks
 //   hs      HS_BLOCKS x N double   score-entropy partial column sums
 // The layout depends on the problem size, so one call's flags can lie where
@@ -84,14 +84,9 @@ inline WsLayout ws_layout(int64_t T, int32_t K, int32_t N, int32_t n_slots) {
     w.flags = off + sizeof(ScanCtl);
     w.ctl_bytes = sizeof(ScanCtl) + sizeof(uint32_t) * (size_t)w.nblk;
     off += align256(w.ctl_bytes);
-    // the chain-free kernel's count words: n_slots rows of one word per block
-    // of (at least) 1024 assignments, rows rounded to 16-byte vectors; they
-    // share the agg and pre regions
-    const int64_t nblk_fine = (A + 1023) / 1024 < 1 ? 1 : (A + 1023) / 1024;
-    const size_t words = (size_t)n_slots * (size_t)((nblk_fine + 3) & ~int64_t(3));
-    const size_t agg_bytes = sizeof(int32_t) * cells > sizeof(int32_t) * words ? sizeof(int32_t) * cells
-                                                                                : sizeof(int32_t) * words;
-    w.agg = off;         off += align256(agg_bytes);
+    // (the chain-free kernel's count words, one per block of >= 2048
+    // assignments and slot, fit the agg region)
+    w.agg = off;         off += align256(sizeof(int32_t) * cells);
     w.pre = off;         off += align256(sizeof(int32_t) * cells);
     w.hs_partial = off;  off += align256(sizeof(double) * (size_t)HS_BLOCKS * (size_t)(N > 0 ? N : 1));
     w.total = off;

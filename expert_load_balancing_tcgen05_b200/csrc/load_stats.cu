@@ -200,6 +200,21 @@ constexpr uint32_t FLAG_AGG = 1, FLAG_PREFIX = 2;
 // slot < 0 get an unused value.  Call with the whole warp, chunks in order:
 // the leader's atomic returns before the warp-wide shuffle of its result, so
 // a later chunk's atomic on the same slot always sees it.
+// The lanes holding `slot` (bit-sliced ballots), for warp_slot_rank and the
+// chain-free kernel's interleaved chunks.
+__device__ __forceinline__ unsigned slot_peers(int slot, int nbits) {
+    unsigned peers = __ballot_sync(FULL, slot >= 0);
+    if (slot < 0) peers = ~peers;
+#pragma unroll
+    for (int bit = 0; bit < 11; ++bit) {
+        if (bit < nbits) {
+            const unsigned B = __ballot_sync(FULL, (slot >> bit) & 1);
+            peers &= ((slot >> bit) & 1) ? B : ~B;
+        }
+    }
+    return peers;
+}
+
 __device__ __forceinline__ int warp_slot_rank(int slot, int nbits, int32_t* my, int lane) {
     unsigned peers = __ballot_sync(FULL, slot >= 0);
     if (slot < 0) peers = ~peers;
@@ -450,10 +465,11 @@ __global__ void __launch_bounds__(LS_THREADS) load_stats_kernel(
 //     flag: no separate flag and no fence on the normal path (a word without
 //     bit 31 -- zero, or the look-back kernel's counts, which never have it
 //     -- reads as "not yet");
-//  3. each block sums, per slot, the words of ALL earlier blocks (32
-//     independent loads at a time, a bounded re-poll of any word not yet
-//     ready): the count of every earlier assignment in that slot, without
-//     waiting on inclusive prefixes;
+//  3. each block sums, per slot, the words of ALL earlier blocks (laid out
+//     [block][slot], so a warp reads one 128-byte line per earlier block; 32
+//     loads in flight, a bounded re-poll of any word not yet ready): the
+//     count of every earlier assignment in that slot, without waiting on
+//     inclusive prefixes;
 //  4. rank = earlier blocks + earlier warps + within the warp;
 //  5. the last block's sums plus its own counts are the totals: counts,
 //     offsets, statistics.  The last block to finish -- no block reads the
@@ -477,19 +493,6 @@ constexpr uint32_t WORD_READY = 0x80000000u;  // a published per-block count: bi
 constexpr uint32_t WORD_BAD = 0x40000000u;    // the publishing block saw an expert id out of range
 constexpr uint32_t WORD_COUNT = 0x3fffffffu;
 
-__device__ __forceinline__ uint4 ld_relaxed_v4(const uint32_t* p) {
-    uint4 v;
-    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p)
-                 : "memory");
-    return v;
-}
-
-// Row stride (in words) of the per-slot count words: one word per block,
-// rounded up to whole 16-byte vectors.
-__host__ __device__ __forceinline__ int word_stride(int nblk) { return (nblk + 3) & ~3; }
-
 template <int C>
 __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     const int32_t* __restrict__ idx, int64_t A, int K, int N, const int32_t* __restrict__ replica_slot,
@@ -506,18 +509,20 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     int32_t* ex = sm_dyn + LS_WARPS * n_slots;  // [n_slots] earlier-block counts
     int32_t* s_slot = ex + n_slots;             // [BPB] this block's expert ids, then slots
     int32_t* s_rank = s_slot + BPB;             // [BPB] in-warp ranks
+    int32_t* s_rep = s_rank + BPB;              // [N] replica slot of each expert (with replicas)
     __shared__ int s_err;
     __shared__ int s_scan[33];
     __shared__ double s_red[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = block_base + (int)blockIdx.x;  // block_base > 0 only in the bounded-wait self-test
     const bool multi = nblk > 1;
-    const int wstride = word_stride(nblk);  // count words: aggw[slot * wstride + block]
-    const int64_t a0 = (int64_t)b * BPB;
+    const int64_t a0 = (int64_t)b * BPB;  // count words: aggw[block * n_slots + slot]
 
     // the block's expert ids (eight independent loads per thread in flight)
 #pragma unroll 8
     for (int v = tid; v < BPB; v += LS_THREADS) s_slot[v] = a0 + v < A ? __ldg(idx + a0 + v) : -1;
+    if (replica_slot != nullptr)
+        for (int e = tid; e < N; e += LS_THREADS) s_rep[e] = __ldg(replica_slot + e);
     if (tid == 0) s_err = 0;
     for (int i = tid; i < LS_WARPS * n_slots; i += LS_THREADS) wh[i] = 0;
     // the gate epilogue's per-tile histograms (tiles of 128 tokens, aligned to
@@ -552,36 +557,56 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
                         if (e < N) c += __ldg(tq + src) + (has_rep ? 0 : __ldg(tq + N + src));
                         else c += __ldg(tq + N + src);
                     }
-                if (b < nblk - 1) st_relaxed_u32(aggw + (int64_t)e * wstride + b, WORD_READY | (uint32_t)c);
+                if (b < nblk - 1) st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (uint32_t)c);
             }
             tc_agg[j] = c;
         }
     }
     __syncthreads();
 
-    // 1. slots, warp histograms, in-warp stable ranks (one chunk of 32 per step)
+    // 1. slots, warp histograms, in-warp stable ranks: four chunks of 32 per
+    //    step, their ballot chains independent; the leaders' atomics on the
+    //    warp's running histogram are issued in chunk order, so a later
+    //    chunk's atomic on a slot always sees the earlier chunks' counts
     int32_t* my = wh + warp * n_slots;
     const int nbits = n_slots > 1 ? 32 - __clz(n_slots - 1) : 0;
     int bad = 0;
 #pragma unroll 1
-    for (int j = 0; j < C; ++j) {
-        const int li = warp * (C * 32) + j * 32 + lane;
-        const int64_t a = a0 + li;
-        int slot = s_slot[li];
-        if (a < A) {
-            if (slot < 0) {
-                slot = -1;  // dropped by the capacity limit: no slot, rank -1
-            } else if (slot >= N) {
-                bad = 1;
-                slot = -1;
-            } else if (replica_slot != nullptr) {
-                const int r = __ldg(replica_slot + slot);
-                if (r >= 0 && ((a / K) & 1)) slot = r;
-                if (slot >= n_slots) { bad = 1; slot = -1; }
+    for (int j0 = 0; j0 < C; j0 += 4) {
+        int sl[4];
+        unsigned pe[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int li = warp * (C * 32) + (j0 + u) * 32 + lane;
+            const int64_t a = a0 + li;
+            int slot = s_slot[li];
+            if (a < A) {
+                if (slot < 0) {
+                    slot = -1;  // dropped by the capacity limit: no slot, rank -1
+                } else if (slot >= N) {
+                    bad = 1;
+                    slot = -1;
+                } else if (replica_slot != nullptr) {
+                    const int r = s_rep[slot];
+                    if (r >= 0 && ((a / K) & 1)) slot = r;
+                    if (slot >= n_slots) { bad = 1; slot = -1; }
+                }
             }
+            sl[u] = slot;
+            pe[u] = slot_peers(slot, nbits);
         }
-        s_rank[li] = warp_slot_rank(slot, nbits, my, lane);
-        s_slot[li] = slot;
+        int seen[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            seen[u] = 0;
+            if (sl[u] >= 0 && lane == __ffs(pe[u]) - 1) seen[u] = atomicAdd(my + sl[u], __popc(pe[u]));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int li = warp * (C * 32) + (j0 + u) * 32 + lane;
+            s_rank[li] = __shfl_sync(FULL, seen[u], __ffs(pe[u]) - 1) + __popc(pe[u] & lanemask_lt());
+            s_slot[li] = sl[u];
+        }
     }
     if (__any_sync(FULL, bad) && lane == 0) atomicOr(&s_err, 2);
     __syncthreads();
@@ -605,14 +630,14 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
             if (pre_published) {
                 if (tc_agg[j] != run) atomicOr(&s_err, 2);  // the tile histograms do not match the indices
             } else if (multi && b < nblk - 1) {
-                st_relaxed_u32(aggw + (int64_t)e * wstride + b, WORD_READY | (blk_err ? WORD_BAD : 0u) | (uint32_t)run);
+                st_relaxed_u32(aggw + (int64_t)b * n_slots + e, WORD_READY | (blk_err ? WORD_BAD : 0u) | (uint32_t)run);
             }
         }
     }
 
-    // 3. counts of all earlier blocks, per slot: its row of count words, up
-    //    to 64 words (16 vectors) in flight at once
-    constexpr int PV = 16;
+    // 3. counts of all earlier blocks, per slot: a warp reads one 128-byte line
+    //    per earlier block (words [block][slot]), 32 blocks in flight at once
+    constexpr int PB = 32;
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false, pred_bad = false;
 #pragma unroll 1
@@ -620,33 +645,28 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         excl[j] = 0;
         const int e = tid + j * LS_THREADS;
         if (e >= n_slots || b == 0) continue;
-        const uint32_t* row = aggw + (int64_t)e * wstride;
         uint64_t t0 = 0;
         int acc = 0;
-        const int nv = (b + 3) >> 2;  // vectors holding blocks 0 .. b-1
 #pragma unroll 1
-        for (int v0 = 0; v0 < nv; v0 += PV) {
-            uint4 vv[PV];
+        for (int q0 = 0; q0 < b; q0 += PB) {
+            uint32_t w[PB];
 #pragma unroll
-            for (int u = 0; u < PV; ++u) vv[u] = v0 + u < nv ? ld_relaxed_v4(row + 4 * (v0 + u)) : make_uint4(0, 0, 0, 0);
-#pragma unroll 1
-            for (int u = 0; u < PV && v0 + u < nv; ++u) {
-                const int q0 = 4 * (v0 + u);
-                uint32_t w4[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+            // first pass: plain L2 loads (ld.global.cg), all in flight; only a
+            // word not yet ready is re-read with the relaxed loads below
+            for (int u = 0; u < PB; ++u)
+                w[u] = q0 + u < b ? __ldcg(aggw + (int64_t)(q0 + u) * n_slots + e) : WORD_READY;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    if (q0 + k >= b) break;
-                    // bounded re-poll of a word block q0+k has not published yet
-                    while (!(w4[k] & WORD_READY) && !timed_out) {
-                        if (t0 == 0) t0 = globaltimer();
-                        else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
-                        __nanosleep(64);
-                        w4[k] = ld_relaxed_u32(row + q0 + k);
-                    }
-                    if (w4[k] & WORD_READY) {
-                        acc += (int)(w4[k] & WORD_COUNT);
-                        pred_bad |= (w4[k] & WORD_BAD) != 0;
-                    }
+            for (int u = 0; u < PB; ++u) {
+                // bounded re-poll of a word block q0+u has not published yet
+                while (!(w[u] & WORD_READY) && !timed_out) {
+                    if (t0 == 0) t0 = globaltimer();
+                    else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
+                    __nanosleep(64);
+                    w[u] = ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e);
+                }
+                if (w[u] & WORD_READY) {
+                    acc += (int)(w[u] & WORD_COUNT);
+                    pred_bad |= (w[u] & WORD_BAD) != 0;
                 }
             }
         }
@@ -704,8 +724,7 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         __syncthreads();
         if (s_last) {
             __threadfence();
-            uint4* w4 = reinterpret_cast<uint4*>(aggw);
-            for (int64_t i = tid; i < (int64_t)n_slots * (wstride / 4); i += LS_THREADS) w4[i] = make_uint4(0, 0, 0, 0);
+            for (int64_t i = tid; i < (int64_t)(nblk - 1) * n_slots; i += LS_THREADS) aggw[i] = 0u;
             if (tid == 0) {
                 ctl->sticky |= ctl->err;
                 ctl->err = 0;
@@ -855,16 +874,16 @@ cudaError_t launch_load_stats(const int32_t* idx, int64_t T, int K, int N, const
     // the smallest blocks (1024, 2048, 4096 or 8192 assignments) that still
     // fit one block per SM, or, beyond that, up to V2_MAX_BLOCKS blocks of 8192
     int chunks = 32;
-    for (int c = 4; c <= 32; c *= 2)
+    for (int c = 8; c <= 32; c *= 2)
         if (A <= (int64_t)V2_WAVE * LS_THREADS * c) { chunks = c; break; }
     const int64_t nb2 = (A + (int64_t)LS_THREADS * chunks - 1) / ((int64_t)LS_THREADS * chunks);
     if (nb2 <= V2_MAX_BLOCKS) {
         const int nb = nb2 < 1 ? 1 : (int)nb2;
         uint32_t* aggw = reinterpret_cast<uint32_t*>(agg);  // one ready-flagged count word per (block, slot)
-        auto kern = chunks == 4 ? load_stats_v2_kernel<4>
-                                : (chunks == 8 ? load_stats_v2_kernel<8>
-                                               : (chunks == 16 ? load_stats_v2_kernel<16> : load_stats_v2_kernel<32>));
-        const size_t lsm2 = lsm + sizeof(int32_t) * 2 * (size_t)LS_THREADS * chunks;  // + ids/slots and ranks
+        auto kern = chunks == 8 ? load_stats_v2_kernel<8>
+                                : (chunks == 16 ? load_stats_v2_kernel<16> : load_stats_v2_kernel<32>);
+        // + ids/slots, ranks and the replica map
+        const size_t lsm2 = lsm + sizeof(int32_t) * (2 * (size_t)LS_THREADS * chunks + (size_t)N);
         if (lsm2 > 48 * 1024) {
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm2);
             if (e != cudaSuccess) return e;
@@ -905,7 +924,7 @@ cudaError_t run_lookback_timeout_probe(void* ws, int32_t* err_out, cudaStream_t 
         // cleared by every call's last block)
         cudaError_t e = cudaMemsetAsync(ctl, 0, 4 * sizeof(int32_t), st);
         if (e != cudaSuccess) return e;
-        const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8 + (probe == 1 ? sizeof(int32_t) * 2 * LS_BLOCK : 0);
+        const size_t smem = sizeof(int32_t) * (LS_WARPS + 1) * 8 + (probe == 1 ? sizeof(int32_t) * (2 * LS_BLOCK + 8) : 0);
         if (probe == 0)
             load_stats_kernel<<<1, LS_THREADS, smem, st>>>(
                 nullptr, 0, 1, 8, nullptr, 8, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, ctl,

@@ -19,7 +19,7 @@
 // call epoch) reset when its last block finishes, but a call must not depend
 // on the previous one having ended cleanly, so every call here first clears,
 // on its own stream, the control block, look-back flags and per-block count
-// words of its layout (about 1.8 MB for the largest workload here).  Two calls whose kernels overlap on the GPU race on the
+// words of its layout (about 1.2 MB for the largest workload here).  Two calls whose kernels overlap on the GPU race on the
 // array; the caller must serialise them.
 #include <mutex>
 
@@ -75,7 +75,7 @@ extern "C" moe_status moe_load_stats_noalloc(const int32_t* topk_idx, int64_t T,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // the control block, the look-back flags and the per-block count words
     // start at zero: the epoch restarts at 0 and no word carries its tag
-    // (about 1.8 MB for the largest workload here)
+    // (about 1.2 MB for the largest workload here)
     const moe::WsLayout L = moe::ws_layout(T, K, N, n_slots);
     if (cudaMemsetAsync(static_cast<char*>(ws) + L.ctl, 0, L.hs_partial - L.ctl, st) != cudaSuccess)
         return MOE_ERR_CUDA;

@@ -370,7 +370,7 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
  *  - Returns MOE_ERR_UNSUPPORTED, enqueuing nothing, when the problem needs
  *    more scratch than that (moe_workspace_bytes(T, K, N, n_slots) larger
  *    than MOE_NOALLOC_SCRATCH_BYTES, 4 MiB; the largest routing workload
- *    here, T = 131072 tokens, K = 8, 288 slots, needs 2,296,320 bytes).
+ *    here, T = 131072 tokens, K = 8, 288 slots, needs 1,706,496 bytes).
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it for the life of the process; make
  *    that first call before any stream capture.  The cached address does
@@ -379,7 +379,7 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
  *  - All calls share the one array, which keeps the last call's contents.
  *    Every call first clears, on its stream, the part that must start at
  *    zero (the scan's control words, look-back flags and per-block count
- *    words: at most about 1.8 MB for the largest workload here), so a call never depends on how the
+ *    words: at most about 1.2 MB for the largest workload here), so a call never depends on how the
  *    previous one ended.  Calls whose kernels
  *    overlap on the GPU -- different streams, or threads, using the same
  *    device -- race on the array: the caller must serialise them.
