@@ -514,13 +514,13 @@ def run_kernel_report(only=None):
     """Per-call device times of the library on every workload (3 warm-up
     calls, then 10 calls captured in a CUDA graph and replayed under CUDA
     events), each against its bound: HBM
-    bytes over the measured copy bandwidth, or the gate's flops over the
-    measured bf16 peak if longer.  Prints a markdown table (not the
+    bytes over the copy bandwidth, or the gate's flops over the bf16 burst
+    peak if longer (the measured peaks when present, else the fallback).  Prints a markdown table (not the
     benchmark's JSON line)."""
     import torch
     from expert_load_balancing_tcgen05_b200 import moe
     from expert_load_balancing_tcgen05_b200 import workloads as W
-    hbm, tf_burst, _, _ = _peaks()
+    hbm, tf_burst, _, peak_kind = _peaks()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
 
@@ -642,7 +642,7 @@ def run_kernel_report(only=None):
     print("|---|---|---|---|---|---|---|")
     for r in rows:
         print(f"| {r[0]} | {r[1]} | {r[2]} | {r[3]:.1f} | {r[4]:.1f} | {r[5]:.2f} | {r[6]} |")
-    print(f"\nbounds: HBM {hbm} GB/s (measured copy), bf16 {tf_burst} TFLOP/s (measured burst)")
+    print(f"\nbounds: HBM {hbm} GB/s (copy), bf16 {tf_burst} TFLOP/s (burst): {peak_kind} peaks")
 
 
 def _cpu_model():
