@@ -11,7 +11,7 @@
 //
 // Design (one CTA per SM, persistent over 128-token tiles):
 //   warp 0      TMA producer: x tile [128 x 64] and the whole W slice
-//               [N x 64] per k-step into a STAGES-deep ring of 128B-swizzled
+//               [N x 64] per k-block into a ring of 128B-swizzled
 //               shared-memory buffers (no multicast).
 //   warp 1      allocates TMEM (2 x N fp32 columns: double-buffered
 //               accumulators) and issues tcgen05.mma.cta_group::1.kind::f16
@@ -38,7 +38,7 @@ constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
 constexpr int EPI_WARPS = 8;             // two per TMEM lane quarter, each owning half the columns
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
-constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
+constexpr uint32_t A_KB_BYTES = BM * BK * 2;  // one k-block of the x tile
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -160,15 +160,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 
 template <int BN>
 struct Cfg {
-    static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
-    static constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;
-    static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    // a ring slot holds KPS consecutive k-blocks (fewer, larger waits and
+    // commits per MMA; the x rows come in 256-byte runs); 192 KB of ring
+    static constexpr int KPS = BN >= 256 ? 1 : 2;
+    static constexpr int STAGES = (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8)) / KPS;
+    static constexpr uint32_t B_KB_BYTES = BN * BK * 2;
+    static constexpr uint32_t KB_BYTES = A_KB_BYTES + B_KB_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;  // 128, 256 or 512: powers of two
     // epilogue exchange (per token row): 2 x 2 reduction floats, up to 8 group
     // scores, one 8-entry candidate list (key, score, index); the wait
     // verdicts; the tile's expert histogram by token parity (2 x BN counts)
     static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8) * 4 + 2 * EPI_WARPS * 4 + 2 * BN * 4;
-    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * KPS * KB_BYTES +
                                          8 * (2 * STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
 
@@ -386,12 +389,12 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
                                                              const __grid_constant__ CUtensorMap tmB, int d,
                                                              const Epi p, int32_t* err, int num_tiles) {
     using C = Cfg<BN>;
-    constexpr int STAGES = C::STAGES;
+    constexpr int STAGES = C::STAGES, KPS = C::KPS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + (size_t)STAGES * A_STAGE_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * C::STAGE_BYTES);
+    uint8_t* sA = smem;                                          // [STAGES * KPS][128 x 64] bf16
+    uint8_t* sB = smem + (size_t)STAGES * KPS * A_KB_BYTES;      // [STAGES * KPS][BN x 64] bf16
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * KPS * C::KB_BYTES);
     // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
@@ -441,12 +444,18 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; kb += KPS, ++it) {
+                    const int nk = min(KPS, num_kb - kb);
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
-                    mbar_expect_tx(full0 + 8 * s, C::STAGE_BYTES);
-                    tma_load_2d(smem_u32(sA + (size_t)s * A_STAGE_BYTES), &tmA, kb * BK, tile * BM, full0 + 8 * s);
-                    tma_load_2d(smem_u32(sB + (size_t)s * C::B_STAGE_BYTES), &tmB, kb * BK, 0, full0 + 8 * s);
+                    mbar_expect_tx(full0 + 8 * s, nk * C::KB_BYTES);
+#pragma unroll
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        tma_load_2d(smem_u32(sA + slot * A_KB_BYTES), &tmA, (kb + j) * BK, tile * BM, full0 + 8 * s);
+                        tma_load_2d(smem_u32(sB + slot * C::B_KB_BYTES), &tmB, (kb + j) * BK, 0, full0 + 8 * s);
+                    }
                 }
             }
             // drain: the last load issued into each ring slot has landed
@@ -466,16 +475,22 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
                 if (!mbar_wait(tempty0 + 8 * a, aph ^ 1, err)) { ok = false; break; }
                 fence_after();
                 const uint32_t d_tmem = tmem_base + a * BN;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; kb += KPS, ++it) {
+                    const int nk = min(KPS, num_kb - kb);
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!mbar_wait(full0 + 8 * s, ph, err)) { ok = false; break; }
                     fence_after();
-                    const uint32_t a_addr = smem_u32(sA + (size_t)s * A_STAGE_BYTES);
-                    const uint32_t b_addr = smem_u32(sB + (size_t)s * C::B_STAGE_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(d_tmem, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc<BN>(),
-                                 (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        const uint32_t a_addr = smem_u32(sA + slot * A_KB_BYTES);
+                        const uint32_t b_addr = smem_u32(sB + slot * C::B_KB_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16(d_tmem, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc<BN>(),
+                                     (kb + j > 0 || k > 0) ? 1u : 0u);
+                    }
                     mma_commit(empty0 + 8 * s);
                 }
                 if (ok) mma_commit(tfull0 + 8 * a);
@@ -528,20 +543,22 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
 // Two-SM variant (N = 256): a cluster of two CTAs computes a 256-token tile
 // with tcgen05.mma.cta_group::2 (M = 256 across the pair, N = 256).  Each CTA
 // loads its own 128 token rows of x and its own half (128 experts) of W per
-// k-step, so a stage is 32 KB per SM instead of 48 KB: half the W traffic
-// from L2 and a third less shared-memory traffic per MMA, with six stages in
-// flight.  The leader CTA (rank 0) owns the full barriers (both CTAs' TMA
+// k-block, 32 KB per SM instead of 48 KB: half the W traffic from L2 and a
+// third less shared-memory traffic per MMA.  The ring has three slots of two
+// k-blocks each (64 KB per slot): one wait, eight MMAs and one commit per
+// slot, and each token row arrives in 256-byte runs.  The leader CTA (rank 0) owns the full barriers (both CTAs' TMA
 // loads complete on them), issues the MMAs, and multicasts its commits to
 // both CTAs' barriers; each CTA's TMEM receives its own 128 rows x 256
 // columns and each CTA runs the same epilogue on them.
 // ===========================================================================
-constexpr int PAIR_STAGES = 6;
-constexpr uint32_t PAIR_STAGE_BYTES = 2u * BM * BK * 2;  // A rows + B half, per CTA
+constexpr int PAIR_KPS = 2;                              // k-blocks per ring slot
+constexpr int PAIR_STAGES = 3;
+constexpr uint32_t PAIR_KB_BYTES = 2u * BM * BK * 2;     // one k-block of A rows + B half, per CTA
 struct PairCfg {
     static constexpr int BN = 256;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr size_t XCH_BYTES = Cfg<256>::XCH_BYTES;
-    static constexpr size_t SMEM_BYTES = 1024 + (size_t)PAIR_STAGES * PAIR_STAGE_BYTES +
+    static constexpr size_t SMEM_BYTES = 1024 + (size_t)PAIR_STAGES * PAIR_KPS * PAIR_KB_BYTES +
                                          8 * (2 * PAIR_STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
 
@@ -607,12 +624,12 @@ template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gate_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int d,
                         const Epi p, int32_t* err, int num_pairs) {
-    constexpr int BN = 256, STAGES = PAIR_STAGES;
+    constexpr int BN = 256, STAGES = PAIR_STAGES, KPS = PAIR_KPS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;                                      // [STAGES][128 x 64] bf16, 128B swizzle
-    uint8_t* sB = smem + (size_t)STAGES * (BM * BK * 2);     // [STAGES][128 x 64] bf16 (this CTA's experts)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * PAIR_STAGE_BYTES);
+    uint8_t* sA = smem;                                          // [STAGES * KPS][128 x 64] bf16, 128B swizzle
+    uint8_t* sB = smem + (size_t)STAGES * KPS * A_KB_BYTES;      // [STAGES * KPS][128 x 64] bf16 (this CTA's experts)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * KPS * PAIR_KB_BYTES);
     // bars: full[STAGES] (leader), empty[STAGES], tfull[2], tempty[2] (leader), done (leader)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
@@ -666,13 +683,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             bool ok = true;
             for (int tp = cluster; tp < num_pairs && ok; tp += nclusters) {
                 const int m0 = tp * 2 * BM + (int)rank * BM;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; kb += KPS, ++it) {
+                    const int nk = min(KPS, num_kb - kb);
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
                     const uint32_t fb = map_to(full0 + 8 * s, 0);
-                    if (leader) mbar_expect_tx(full0 + 8 * s, 2 * PAIR_STAGE_BYTES);
-                    tma_load_2d_pair(smem_u32(sA + (size_t)s * (BM * BK * 2)), &tmA, kb * BK, m0, fb);
-                    tma_load_2d_pair(smem_u32(sB + (size_t)s * (BM * BK * 2)), &tmB, kb * BK, (int)rank * BM, fb);
+                    if (leader) mbar_expect_tx(full0 + 8 * s, 2 * nk * PAIR_KB_BYTES);
+#pragma unroll
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        tma_load_2d_pair(smem_u32(sA + slot * A_KB_BYTES), &tmA, (kb + j) * BK, m0, fb);
+                        tma_load_2d_pair(smem_u32(sB + slot * A_KB_BYTES), &tmB, (kb + j) * BK, (int)rank * BM, fb);
+                    }
                 }
             }
             // drain: this CTA's last loads into each slot have landed (the leader sees all of them)
@@ -694,16 +717,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (!mbar_wait(tempty0 + 8 * a, aph ^ 1, err)) { ok = false; break; }
                 fence_after();
                 const uint32_t d_tmem = tmem_base + a * BN;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; kb += KPS, ++it) {
+                    const int nk = min(KPS, num_kb - kb);
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!mbar_wait(full0 + 8 * s, ph, err)) { ok = false; break; }
                     fence_after();
-                    const uint32_t a_addr = smem_u32(sA + (size_t)s * (BM * BK * 2));
-                    const uint32_t b_addr = smem_u32(sB + (size_t)s * (BM * BK * 2));
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16_pair(d_tmem, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc_pair(),
-                                      (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        const uint32_t a_addr = smem_u32(sA + slot * A_KB_BYTES);
+                        const uint32_t b_addr = smem_u32(sB + slot * A_KB_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16_pair(d_tmem, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc_pair(),
+                                          (kb + j > 0 || k > 0) ? 1u : 0u);
+                    }
                     mma_commit_pair(empty0 + 8 * s);
                 }
                 if (ok) mma_commit_pair(tfull0 + 8 * a);

@@ -66,6 +66,9 @@ TC_CASES = [
     ("collapse", 300, 7168),         # celebrity logit offsets
     ("prefill_replicas", 260, 7168),  # Zipf logit offsets
     ("softmax_dispatch", 389, 4096),  # N=128 softmax
+    # odd k-block counts: the last ring slot holds one k-block of two
+    ("v3_router", 300, 936),         # 15 k-blocks (14*64 + 40), pair kernel
+    ("softmax_dispatch", 257, 264),  # 5 k-blocks, N=128 one-SM kernel
 ]
 
 
@@ -77,6 +80,7 @@ def test_gate_tc_against_oracle(orc, name, T, d):
 def test_gate_tc_n64_sigmoid(orc):
     wl = W.Workload("n64", 0, 0, 0, 64, 6, fn=1, n_groups=4, topk_groups=2, scale=1.0, has_bias=True)
     _run_and_check(orc, wl, 700, 512, seed=3)
+    _run_and_check(orc, wl, 333, 192, seed=4)  # 3 k-blocks: an odd count
 
 
 def test_gate_tc_many_tiles_per_cta(orc):
