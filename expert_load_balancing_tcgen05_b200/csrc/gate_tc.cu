@@ -168,9 +168,10 @@ struct Cfg {
     static constexpr uint32_t KB_BYTES = A_KB_BYTES + B_KB_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;  // 128, 256 or 512: powers of two
     // epilogue exchange (per token row): 2 x 2 reduction floats, up to 8 group
-    // scores, one 8-entry candidate list (key, score, index); the wait
+    // scores and 8 group second-largest keys, one 8-entry candidate list
+    // (key, score, index); the wait
     // verdicts; the tile's expert histogram by token parity (2 x BN counts)
-    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8) * 4 + 2 * EPI_WARPS * 4 + 2 * BN * 4;
+    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8 + 8) * 4 + 2 * EPI_WARPS * 4 + 2 * BN * 4;
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * KPS * KB_BYTES +
                                          8 * (2 * STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
@@ -211,6 +212,7 @@ struct Xch {
     int* li;      // [BM][8]
     int* agree;   // [2][EPI_WARPS]: per tile parity, each warp's wait verdict
     int* hist;    // [2][BN]: the tile's chosen experts counted by token parity (fused, tile_counts given)
+    float* gt2;   // [BM][8]: each group's second-largest key
 };
 
 // One token row (this thread's TMEM lane) of one finished tile.  The two
@@ -244,6 +246,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                     if (key > t1) { t2 = t1; t1 = key; } else if (key > t2) { t2 = key; }
                 }
                 x.gs[row * 8 + c] = p.group_topn == 1 ? t1 : __fadd_rn(t1, t2);
+                x.gt2[row * 8 + c] = t2;
                 if (srow) store32(srow + 32 * c, v);
             }
             epi_sync();
@@ -258,20 +261,44 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 for (int c2 = 0; c2 < NC; ++c2) rank += (c2 != c && beats(gs[c2], c2, gs[c], c)) ? 1 : 0;
                 if (rank < p.topk_groups) keep |= 1u << c;
             }
+            // A lower bound on the row's K-th best kept key: every kept group
+            // holds two keys at or above its second largest, so with
+            // 2 * topk_groups >= K the K best keys are all at or above the
+            // smallest kept second-largest key.  Only those candidates are
+            // offered (lanes are token rows with different kept groups, so
+            // offering every kept column would run every column in every warp).
+            float t0 = INFINITY;
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+                if ((keep >> c) & 1u) t0 = fminf(t0, x.gt2[row * 8 + c]);
+            if (2 * p.topk_groups < p.K || !(t0 < INFINITY)) t0 = -INFINITY;
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
                 const bool kc = (keep >> c) & 1u;
+                if (!__any_sync(0xffffffffu, kc)) continue;
 #pragma unroll 1
                 for (int q = 0; q < 4; ++q) {
-                    float v8[8];
+                    float v8[8], k8[8];
                     tmem_ld8(taddr + 32 * c + 8 * q, v8);  // warp-collective: every lane loads every piece
-                    if (kc) {
+                    unsigned m = 0;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int col = 32 * c + 8 * q + i;
-                            const float sv = sigmoid_f(v8[i] + off_s[col]);
-                            top.offer(__fadd_rn(sv, bias_s[col]), col, sv);
+                    for (int i = 0; i < 8; ++i) {
+                        const int col = 32 * c + 8 * q + i;
+                        v8[i] = sigmoid_f(v8[i] + off_s[col]);
+                        k8[i] = __fadd_rn(v8[i], bias_s[col]);
+                        if (kc && !(k8[i] < t0)) m |= 1u << i;  // a NaN key is offered, as without the bound
+                    }
+                    // survivors in ascending column order, one per lane per round
+                    while (__any_sync(0xffffffffu, m != 0)) {
+                        if (m != 0) {
+                            const int i = __ffs(m) - 1;
+                            m &= m - 1;
+                            float kk = k8[0], sv = v8[0];
+#pragma unroll
+                            for (int j = 1; j < 8; ++j)
+                                if (i == j) { kk = k8[j]; sv = v8[j]; }
+                            top.offer(kk, 32 * c + 8 * q + i, sv);
                         }
                     }
                 }
@@ -407,6 +434,7 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
     xch.agree = xch.li + 8 * BM;
     xch.hist = xch.agree + 2 * EPI_WARPS;
+    xch.gt2 = reinterpret_cast<float*>(xch.hist + 2 * BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
@@ -642,6 +670,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
     xch.agree = xch.li + 8 * BM;
     xch.hist = xch.agree + 2 * EPI_WARPS;
+    xch.gt2 = reinterpret_cast<float*>(xch.hist + 2 * BN);
     for (int i = threadIdx.x; i < 2 * BN; i += blockDim.x) xch.hist[i] = 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

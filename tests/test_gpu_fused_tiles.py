@@ -143,3 +143,33 @@ def test_route_tiles_rejects_what_the_epilogue_cannot_select():
     with pytest.raises(moe.MoeError) as e:
         moe.moe_route_tiles(cfg, inp["x"], inp["W"], None, inp["bias"], idx, w, tiles, ws)  # K = 16 > 8
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kind", ["zero_gate", "twin_experts", "quad_experts_topn1"])
+def test_route_tiles_with_ties_match_oracle(orc, monkeypatch, kind):
+    """Tied keys inside and across groups: the epilogue's candidate bound
+    admits keys equal to it and the choice keeps (key desc, index asc).
+    zero_gate: every score is 0.5 and every key equal without bias;
+    twin_experts / quad_experts: experts share their gate row (and bias)
+    in pairs or fours, so every key has equal partners."""
+    wl = W.WORKLOADS["v3_router"].with_(T=1500, d=512)
+    if kind == "quad_experts_topn1":
+        wl = wl.with_(group_topn=1)
+    inp = W.make_inputs(wl, device="cuda", seed=41)
+    if kind == "zero_gate":
+        inp["W"] = torch.zeros_like(inp["W"])
+        inp["bias"] = None
+    else:
+        m = 2 if kind == "twin_experts" else 4
+        src = torch.arange(wl.N, device="cuda") // m * m
+        inp["W"] = inp["W"][src].contiguous()
+        inp["bias"] = inp["bias"][src].contiguous()
+    idx, w, tiles, _ = _fused(wl, inp)
+    s = _scores_only(wl, inp, monkeypatch)
+    b = inp["bias"].cpu().numpy() if inp["bias"] is not None else None
+    ri, rw = orc.select(to_np(s), b, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+    assert np.array_equal(to_np(idx), ri)
+    assert np.array_equal(to_np(w), rw)
+    assert np.array_equal(to_np(tiles), _tile_hist_ref(ri, wl.N))
+    if kind == "zero_gate":
+        assert np.array_equal(ri, np.broadcast_to(np.arange(wl.K, dtype=ri.dtype), ri.shape))
