@@ -165,7 +165,10 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, bool tot_share
     }
     if (lane == 0) { s_red[warp] = mx; s_red[8 + warp] = var; s_red[16 + warp] = H; s_red[24 + warp] = Hs; }
     __syncthreads();
-    if (tid == 0) {
+    if (tid < 4) {
+        // the warps' partials in the same order in every thread; the fields
+        // are split over four threads so the divisions and the square root
+        // do not run one after another
         double rmx = s_red[0], rvar = 0.0, rH = 0.0, rHs = 0.0;
         for (int w = 0; w < LS_WARPS; ++w) {
             rmx = fmax(rmx, s_red[w]);
@@ -173,19 +176,24 @@ __device__ __forceinline__ void finish_totals(const int32_t* tot, bool tot_share
             rH += s_red[16 + w];
             rHs += s_red[24 + w];
         }
-        rvar /= (double)(n_slots > 0 ? n_slots : 1);
-        const int err = (err_word != nullptr ? ld_volatile(err_word) : 0) | local_err;
-        stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
-        stats->n_slots = n_slots;
-        stats->total = (int64_t)total_i;
-        stats->max_load = (int64_t)rmx;
-        stats->mean = mean;
-        stats->imbalance = mean > 0.0 ? rmx / mean : 0.0;
-        stats->std_over_mean = mean > 0.0 ? sqrt(rvar) / mean : 0.0;
-        stats->entropy_load_bits = rH;
-        stats->entropy_score_bits = hs_partial != nullptr ? rHs : NAN;
-        stats->capacity_fixed = rmx * (double)n_slots;
-        stats->capacity_125 = 1.25 * mean;
+        if (tid == 0) {
+            const int err = (err_word != nullptr ? ld_volatile(err_word) : 0) | local_err;
+            stats->status = err == 0 ? MOE_OK : ((err & 1) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID);
+            stats->n_slots = n_slots;
+            stats->total = (int64_t)total_i;
+            stats->max_load = (int64_t)rmx;
+            stats->mean = mean;
+        } else if (tid == 1) {
+            stats->imbalance = mean > 0.0 ? rmx / mean : 0.0;
+            stats->capacity_fixed = rmx * (double)n_slots;
+            stats->capacity_125 = 1.25 * mean;
+        } else if (tid == 2) {
+            rvar /= (double)(n_slots > 0 ? n_slots : 1);
+            stats->std_over_mean = mean > 0.0 ? sqrt(rvar) / mean : 0.0;
+        } else {
+            stats->entropy_load_bits = rH;
+            stats->entropy_score_bits = hs_partial != nullptr ? rHs : NAN;
+        }
     }
 }
 
@@ -636,8 +644,9 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
     }
 
     // 3. counts of all earlier blocks, per slot: a warp reads one 128-byte line
-    //    per earlier block (words [block][slot]), 32 blocks in flight at once
-    constexpr int PB = 32;
+    //    per earlier block (words [block][slot]), up to 64 blocks in flight at
+    //    once; the words not ready yet are re-read together, round by round
+    constexpr int PB = 64;
     int excl[LS_SLOTS_PER_THREAD];
     bool timed_out = false, pred_bad = false;
 #pragma unroll 1
@@ -655,15 +664,24 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
             // word not yet ready is re-read with the relaxed loads below
             for (int u = 0; u < PB; ++u)
                 w[u] = q0 + u < b ? __ldcg(aggw + (int64_t)(q0 + u) * n_slots + e) : WORD_READY;
+            bool pending = false;
+#pragma unroll
+            for (int u = 0; u < PB; ++u) pending |= !(w[u] & WORD_READY);
+            // bounded rounds: every word not ready yet is re-read (all in
+            // flight), until each is ready or the wait limit has passed
+            while (pending && !timed_out) {
+                if (t0 == 0) t0 = globaltimer();
+                else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
+                __nanosleep(64);
+#pragma unroll
+                for (int u = 0; u < PB; ++u)
+                    if (!(w[u] & WORD_READY)) w[u] = ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e);
+                pending = false;
+#pragma unroll
+                for (int u = 0; u < PB; ++u) pending |= !(w[u] & WORD_READY);
+            }
 #pragma unroll
             for (int u = 0; u < PB; ++u) {
-                // bounded re-poll of a word block q0+u has not published yet
-                while (!(w[u] & WORD_READY) && !timed_out) {
-                    if (t0 == 0) t0 = globaltimer();
-                    else if (globaltimer() - t0 > WAIT_LIMIT_NS) { timed_out = true; break; }
-                    __nanosleep(64);
-                    w[u] = ld_relaxed_u32(aggw + (int64_t)(q0 + u) * n_slots + e);
-                }
                 if (w[u] & WORD_READY) {
                     acc += (int)(w[u] & WORD_COUNT);
                     pred_bad |= (w[u] & WORD_BAD) != 0;
@@ -724,7 +742,11 @@ __global__ void __launch_bounds__(LS_THREADS, 1) load_stats_v2_kernel(
         __syncthreads();
         if (s_last) {
             __threadfence();
-            for (int64_t i = tid; i < (int64_t)(nblk - 1) * n_slots; i += LS_THREADS) aggw[i] = 0u;
+            // (the region starts 256-byte aligned: 16-byte stores, then the tail)
+            const int64_t nw = (int64_t)(nblk - 1) * n_slots;
+            uint4* aw4 = reinterpret_cast<uint4*>(aggw);
+            for (int64_t i = tid; i < nw / 4; i += LS_THREADS) aw4[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int64_t i = (nw / 4) * 4 + tid; i < nw; i += LS_THREADS) aggw[i] = 0u;
             if (tid == 0) {
                 ctl->sticky |= ctl->err;
                 ctl->err = 0;
