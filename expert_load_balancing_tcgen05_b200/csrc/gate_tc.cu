@@ -169,9 +169,13 @@ struct Cfg {
     static constexpr int TMEM_COLS = 2 * BN;  // 128, 256 or 512: powers of two
     // epilogue exchange (per token row): 2 x 2 reduction floats, up to 8 group
     // scores and 8 group second-largest keys, one 8-entry candidate list
-    // (key, score, index); the wait
-    // verdicts; the tile's expert histogram by token parity (2 x BN counts)
-    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8 + 3 * 8 + 8) * 4 + 2 * EPI_WARPS * 4 + 2 * BN * 4;
+    // (key, score, index); the wait verdicts; the tile's expert histogram by
+    // token parity (2 x BN counts).  The scores-only epilogue uses the space
+    // of the lists, histogram and second-largest keys as its store staging.
+    static constexpr size_t XCH_LISTS = (size_t)BM * (3 * 8 + 8) * 4 + 2 * BN * 4;
+    static constexpr size_t XCH_STAGE = (size_t)EPI_WARPS * 32 * 20 * 4;
+    static constexpr size_t XCH_BYTES = (size_t)BM * (4 + 8) * 4 + 2 * EPI_WARPS * 4 + 16 +
+                                        (XCH_LISTS > XCH_STAGE ? XCH_LISTS : XCH_STAGE);
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * KPS * KB_BYTES +
                                          8 * (2 * STAGES + 5) + 16 + 2 * 4 * BN + XCH_BYTES;
 };
@@ -213,7 +217,54 @@ struct Xch {
     int* agree;   // [2][EPI_WARPS]: per tile parity, each warp's wait verdict
     int* hist;    // [2][BN]: the tile's chosen experts counted by token parity (fused, tile_counts given)
     float* gt2;   // [BM][8]: each group's second-largest key
+    float* stage;  // [EPI_WARPS][32][20], 16-byte aligned: scores-only epilogue, aliases lk..gt2
 };
+
+// The exchange, carved from shared memory at `base` (4-byte aligned).
+template <int BN>
+__device__ __forceinline__ Xch carve_xch(float* base) {
+    Xch x;
+    x.red = base;
+    x.gs = x.red + 4 * BM;
+    x.agree = reinterpret_cast<int*>(x.gs + 8 * BM);
+    float* q = reinterpret_cast<float*>(x.agree + 2 * EPI_WARPS);
+    q = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(q) + 15) & ~uintptr_t(15));
+    x.lk = q;
+    x.ls = x.lk + 8 * BM;
+    x.li = reinterpret_cast<int*>(x.ls + 8 * BM);
+    x.hist = x.li + 8 * BM;
+    x.gt2 = reinterpret_cast<float*>(x.hist + 2 * BN);
+    x.stage = q;
+    return x;
+}
+
+// One 32-column chunk of scores for the warp's 32 consecutive token rows
+// (this lane's row in v), written through the warp's [32][20] staging tile
+// 16 columns at a time: each store instruction then writes 64 contiguous
+// bytes of 8 rows, not 16 bytes of 32 rows (a quarter of the L2 write
+// requests).  Rows at or past T are not written.
+template <int BN>
+__device__ __forceinline__ void store_chunk_staged(const Epi& p, int64_t grow, int c, const float (&v)[32],
+                                                   float* stage, int lane) {
+    const int64_t r0 = grow - lane;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float* mine = stage + lane * 20;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4*>(mine + 4 * q) =
+                make_float4(v[16 * hh + 4 * q], v[16 * hh + 4 * q + 1], v[16 * hh + 4 * q + 2], v[16 * hh + 4 * q + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + (lane >> 2), cq = lane & 3;
+            const float4 val = *reinterpret_cast<const float4*>(stage + r * 20 + 4 * cq);
+            if (r0 + r < (int64_t)p.T)
+                *reinterpret_cast<float4*>(p.scores + (r0 + r) * BN + 32 * c + 16 * hh + 4 * cq) = val;
+        }
+        __syncwarp();
+    }
+}
 
 // One token row (this thread's TMEM lane) of one finished tile.  The two
 // warps of a lane quarter split the columns: half h owns chunks
@@ -226,6 +277,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                                              const float* off_s, const float* bias_s, const Xch& x) {
     constexpr int NC = BN / 32, NCH = NC / 2;
     const int c_lo = h * NCH;
+    const int lane = threadIdx.x & 31, warp_in_epi = (int)(threadIdx.x >> 5) - 2;  // epilogue warps are 2..
     const bool live = grow < p.T;
     float* srow = (p.scores != nullptr && live) ? p.scores + grow * BN : nullptr;
     float v[32];
@@ -323,7 +375,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
-                if (srow) store32(srow + 32 * c, v);
+                if (p.scores != nullptr) store_chunk_staged<BN>(p, grow, c, v, x.stage + warp_in_epi * (32 * 20), lane);
             }
         }
     } else {
@@ -370,7 +422,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
-                if (srow) store32(srow + 32 * c, v);
+                if (p.scores != nullptr) store_chunk_staged<BN>(p, grow, c, v, x.stage + warp_in_epi * (32 * 20), lane);
             }
         }
     }
@@ -426,15 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1) gate_tc_kernel(const __grid_consta
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
     float* bias_s = off_s + BN;
-    Xch xch;
-    xch.red = bias_s + BN;
-    xch.gs = xch.red + 4 * BM;
-    xch.lk = xch.gs + 8 * BM;
-    xch.ls = xch.lk + 8 * BM;
-    xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
-    xch.agree = xch.li + 8 * BM;
-    xch.hist = xch.agree + 2 * EPI_WARPS;
-    xch.gt2 = reinterpret_cast<float*>(xch.hist + 2 * BN);
+    const Xch xch = carve_xch<BN>(bias_s + BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
@@ -662,15 +706,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
     float* bias_s = off_s + BN;
-    Xch xch;
-    xch.red = bias_s + BN;
-    xch.gs = xch.red + 4 * BM;
-    xch.lk = xch.gs + 8 * BM;
-    xch.ls = xch.lk + 8 * BM;
-    xch.li = reinterpret_cast<int*>(xch.ls + 8 * BM);
-    xch.agree = xch.li + 8 * BM;
-    xch.hist = xch.agree + 2 * EPI_WARPS;
-    xch.gt2 = reinterpret_cast<float*>(xch.hist + 2 * BN);
+    const Xch xch = carve_xch<BN>(bias_s + BN);
     for (int i = threadIdx.x; i < 2 * BN; i += blockDim.x) xch.hist[i] = 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
