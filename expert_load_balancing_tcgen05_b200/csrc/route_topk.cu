@@ -274,12 +274,12 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
         if (t + warps < T) load_row<EPL>(scores + (t + warps) * N, lane, N, nv);
 #pragma unroll
         for (int i = 0; i < EPL; ++i) kv[i] = __fadd_rn(sv[i], b[i]);
-        // 1. the lane's two largest keys
+        // 1. the lane's two largest keys (a NaN key enters neither)
         float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
-            t2 = kv[i] > t1 ? t1 : (kv[i] > t2 ? kv[i] : t2);
-            t1 = kv[i] > t1 ? kv[i] : t1;
+            t2 = fmaxf(t2, fminf(t1, kv[i]));
+            t1 = fmaxf(t1, kv[i]);
         }
         // 2. groups: the group's top two over its lanes, scores, ranks
         bool kept = true;
@@ -308,11 +308,15 @@ __global__ void __launch_bounds__(SW_THREADS, 3) route_select_warp_kernel(
             th_u = __reduce_max_sync(FULL, u2);
             if (u2 == th_u) u2 = 0u;
         }
-        // 4. survivors, compacted in expert order, one per lane
+        // 4. survivors, compacted in expert order, one per lane.  For a key
+        //    that is not NaN, ord_key(k) >= th_u is k >= th_f with th_f the
+        //    float whose image th_u is (-inf when no lane had a value left)
+        const float th_f = th_u == 0u ? -INFINITY
+                                      : __uint_as_float((th_u & 0x80000000u) ? (th_u & 0x7fffffffu) : ~th_u);
         unsigned m = 0;
         if (kept) {
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) m |= (ord_key(kv[i]) >= th_u ? 1u : 0u) << i;
+            for (int i = 0; i < EPL; ++i) m |= (kv[i] >= th_f ? 1u : 0u) << i;
         }
         const int cnt = __popc(m);
         const int total = __reduce_add_sync(FULL, (unsigned)cnt);
