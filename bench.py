@@ -554,6 +554,10 @@ def run_kernel_report(only=None):
     for name in names:
         if only is not None and name != only:
             continue
+        # a short idle gap first: after the large workloads' seconds of full-power
+        # work the clocks take a moment to recover, which the next rows would see
+        torch.cuda.synchronize()
+        time.sleep(2.0)
         wl = W.WORKLOADS[name]
         T, d, N, K = wl.T, wl.d, wl.N, wl.K
         A = T * K
