@@ -11,16 +11,19 @@
 //
 // Design (one CTA per SM, persistent over 128-token tiles):
 //   warp 0      TMA producer: x tile [128 x 64] and the whole W slice
-//               [N x 64] per k-block into a ring of 128B-swizzled
-//               shared-memory buffers (no multicast).
+//               [N x 64] per k-block into a 192 KB ring of 128B-swizzled
+//               shared-memory slots of one or two k-blocks (no multicast).
 //   warp 1      allocates TMEM (2 x N fp32 columns: double-buffered
 //               accumulators) and issues tcgen05.mma.cta_group::1.kind::f16
 //               M=128, N=BN, K=16 from one elected thread; tcgen05.commit
 //               frees ring slots and signals a finished accumulator.
-//   warps 2..5  epilogue: tcgen05.ld rows out of TMEM (thread = token row),
-//               add the logit offset, apply the nonlinearity (softmax has the
-//               whole row in one thread) and store fp32 scores; then release
-//               the accumulator so the next tile's MMAs overlap this work.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, each owning half
+//               the columns: tcgen05.ld rows out of TMEM (thread = token
+//               row), add the logit offset, apply the nonlinearity (softmax
+//               exchanges the halves' max and sum) and store fp32 scores, or
+//               select in place; then release the accumulator so the next
+//               tile's MMAs overlap this work.
+// The N = 256 variant further down runs the same roles on a pair of CTAs.
 // Every barrier wait is bounded: on expiry the kernel records the error in
 // the workspace, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
