@@ -125,7 +125,7 @@ moe_status moe_route(const moe_route_cfg* cfg, const void* x, const void* w_gate
     if (c.T == 0) return MOE_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (x != nullptr) {
-        if (w_gate == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+        if (w_gate == nullptr || ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
         if (c.d <= 0 || c.N > MAX_N) return MOE_ERR_INVALID;
         if (ws_bytes < moe_workspace_bytes(c.T, c.K, c.N, c.N)) return MOE_ERR_INVALID;
         if (c.in_dtype != MOE_F32 && c.in_dtype != MOE_BF16) return MOE_ERR_INVALID;
@@ -155,7 +155,7 @@ moe_status moe_route_tiles(const moe_route_cfg* cfg, const void* x, const void* 
     moe_status s = check_route_cfg(cfg);
     if (s != MOE_OK) return s;
     const moe_route_cfg& c = *cfg;
-    if (x == nullptr || w_gate == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+    if (x == nullptr || w_gate == nullptr || ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
     if (c.T > 0 && (topk_idx == nullptr || topk_w == nullptr || tile_counts == nullptr)) return MOE_ERR_INVALID;
     if (c.d <= 0 || c.in_dtype != MOE_BF16) return c.in_dtype == MOE_F32 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID;
     if (!gate_tc_supported(c.N) || !gate_tc_can_fuse(c.N, c.K, c.score_fn, c.n_groups, c.group_topn))
@@ -177,7 +177,7 @@ moe_status moe_load_stats(const int32_t* topk_idx, int64_t T, int32_t K, int32_t
                           moe_stream_t stream) {
     if (T < 0 || K <= 0 || K > 32 || N <= 0 || n_slots < N || n_slots > MAX_SLOTS) return MOE_ERR_INVALID;
     if (T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
-    if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+    if (counts == nullptr || offsets == nullptr || ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
     if (T > 0 && (topk_idx == nullptr || rank == nullptr)) return MOE_ERR_INVALID;  // empty batch: may be NULL
     if (replica_slot == nullptr && n_slots != N) return MOE_ERR_INVALID;
     if (scores != nullptr && (N > MAX_N || (score_fn != MOE_SOFTMAX && score_fn != MOE_SIGMOID)))
@@ -193,7 +193,7 @@ moe_status moe_load_stats_tiles(const int32_t* topk_idx, int64_t T, int32_t K, i
                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
     if (T < 0 || K <= 0 || K > 32 || N <= 0 || n_slots < N || n_slots > MAX_SLOTS) return MOE_ERR_INVALID;
     if (T * (int64_t)K >= ((int64_t)1 << 31)) return MOE_ERR_INVALID;
-    if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID;
+    if (counts == nullptr || offsets == nullptr || ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
     if (T > 0 && (topk_idx == nullptr || rank == nullptr || tile_counts == nullptr)) return MOE_ERR_INVALID;
     if (replica_slot == nullptr && n_slots != N) return MOE_ERR_INVALID;
     if (ws_bytes < moe_workspace_bytes(T, K, N, n_slots)) return MOE_ERR_INVALID;
@@ -225,7 +225,7 @@ moe_status moe_route_capacity(const moe_route_cfg* cfg, const float* scores, con
     if (capacity < 0) capacity = moe_capacity_limit(c.T, c.K, c.N);  // the page's 1.25 factor
     if (c.T > 0 && (scores == nullptr || topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID;
     if (scores != nullptr && !aligned16(scores)) return MOE_ERR_INVALID;
-    if (ws == nullptr || ws_bytes < moe_capacity_workspace_bytes(c.T, c.K, c.N)) return MOE_ERR_INVALID;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < moe_capacity_workspace_bytes(c.T, c.K, c.N)) return MOE_ERR_INVALID;
     // the counters are always written: to info, or else to the workspace header
     static_assert(sizeof(moe_capacity_info) == 4 * sizeof(long long), "info layout");
     long long* inf = info != nullptr ? reinterpret_cast<long long*>(info)
@@ -305,7 +305,7 @@ moe_status moe_combine(const void* y, int32_t dtype, int64_t T, int32_t d, int32
 }
 
 moe_status moe_workspace_status(void* ws, moe_stream_t stream) {
-    if (ws == nullptr) return MOE_ERR_INVALID;
+    if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     struct {
         WsHeader h;
@@ -332,7 +332,7 @@ moe_status moe_workspace_status(void* ws, moe_stream_t stream) {
 }
 
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, moe_stream_t stream) {
-    if (ws == nullptr || ws_bytes < moe_workspace_bytes(2 * LS_BLOCK, 1, 8, 8)) return MOE_ERR_INVALID;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < moe_workspace_bytes(2 * LS_BLOCK, 1, 8, 8)) return MOE_ERR_INVALID;
     int32_t err = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (run_lookback_timeout_probe(ws, &err, st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -103,7 +103,9 @@ typedef struct {
  * and n_slots histogram slots (n_slots >= N; N + replicas).  One workspace
  * may serve every call on one stream; calls that overlap on the GPU need
  * their own workspaces.  Zero-fill it once before its first use; every call
- * leaves it ready for the next one, so no per-call initialisation is needed. */
+ * leaves it ready for the next one, so no per-call initialisation is needed.
+ * A workspace must start on a 16-byte boundary (the calls that take one
+ * return MOE_ERR_INVALID otherwise). */
 size_t moe_workspace_bytes(int64_t T, int32_t K, int32_t N, int32_t n_slots);
 
 /*
@@ -206,7 +208,8 @@ moe_status moe_route_balanced(int64_t T, int32_t K, int32_t N, float route_scale
  * the page's rule, moe_capacity_limit(T, K, N) = ceil(1.25 * T*K/N).
  * topk_idx, topk_w [T,K] out; info (device, may be NULL) receives the
  * capacity and the overflow / reroute / drop counts.  ws: a zero-filled
- * workspace of moe_capacity_workspace_bytes() bytes, kept between calls.
+ * workspace of moe_capacity_workspace_bytes() bytes, kept between calls,
+ * on a 16-byte boundary.
  * Six launches (candidates, two load-statistics passes, reroute, finalize);
  * every decision comes from stable ranks, so the result equals the
  * sequential walk and is deterministic.

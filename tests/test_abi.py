@@ -204,3 +204,22 @@ def test_route_tiles_and_tile_stats_reject_bad_arguments(moe):
                                   None) == 1  # replica slots without a replica map
     assert L.moe_load_stats_tiles(FAKE, 64, 8, 256, FAKE, None, 256, None, FAKE, FAKE, FAKE, None, FAKE, wsl - 1,
                                   None) == 1
+
+
+def test_workspace_must_be_16_byte_aligned(moe):
+    """Every call that takes a workspace refuses one that does not start on a
+    16-byte boundary, before any launch (all other arguments here are valid)."""
+    L = moe._lib
+    by = ctypes.byref
+    cfg = _cfg(moe)
+    ws = L.moe_workspace_bytes(64, 8, 256, 256)
+    assert L.moe_route(by(cfg), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, MISALIGNED, ws, None) == 1
+    assert L.moe_route_tiles(by(cfg), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, MISALIGNED, ws, None) == 1
+    assert L.moe_load_stats(FAKE, 64, 8, 256, None, 256, None, FAKE, FAKE, FAKE, None, 1, None, MISALIGNED, ws,
+                            None) == 1
+    assert L.moe_load_stats_tiles(FAKE, 64, 8, 256, FAKE, None, 256, None, FAKE, FAKE, FAKE, None, MISALIGNED, ws,
+                                  None) == 1
+    wsc = L.moe_capacity_workspace_bytes(64, 8, 256)
+    assert L.moe_route_capacity(by(cfg), FAKE, None, 5, FAKE, FAKE, None, MISALIGNED, wsc, None) == 1
+    assert L.moe_workspace_status(MISALIGNED, None) == 1
+    assert L.moe_selftest_wait_timeout(MISALIGNED, 1 << 24, None) == 1
