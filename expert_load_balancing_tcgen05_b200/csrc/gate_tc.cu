@@ -849,6 +849,272 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
 }
 
+
+// ===========================================================================
+// Split-K variant for batches with fewer 256-token tiles than CTA pairs:
+// clusters of 2 * S CTAs (S = 2..4 pairs), each taking its tiles one after
+// another.  For every tile, pair p (cluster ranks
+// 2p and 2p + 1, a tcgen05 CTA pair) runs the same producer / MMA roles as the
+// kernel above over its own range of k-blocks into its own TMEM.  Then the
+// pairs p >= 1 copy their accumulators into their idle TMA rings, every
+// thread of the cluster meets at a cluster barrier, and pair 0 adds the other
+// pairs' partial sums (read over distributed shared memory, in pair order, so
+// the result does not depend on timing) into its TMEM and runs the usual
+// epilogue.  No atomics, no waits on other CTAs beyond the cluster barriers,
+// which every thread reaches on every path.
+// ===========================================================================
+// staged partial sums, as float4 pieces [chunk of 32 columns][piece of 4][row]:
+// the 32 rows of a warp's piece are 512 contiguous bytes, so both the staging
+// stores and the remote loads of the fold move whole lines
+__device__ __forceinline__ uint32_t split_piece(int c, int q, int row) { return (uint32_t)((c * 8 + q) * 128 + row); }
+
+__device__ __forceinline__ void mma_commit_pair_mask(uint32_t bar, uint16_t mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(mask)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
+    float4 r;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return r;
+}
+
+template <bool FUSED>
+__global__ void __launch_bounds__(THREADS, 1)
+    gate_tc_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int d,
+                         const Epi p, int32_t* err, int num_pairs, int splits) {
+    constexpr int BN = 256, STAGES = PAIR_STAGES, KPS = PAIR_KPS, NCH = BN / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + (size_t)STAGES * KPS * A_KB_BYTES;
+    float4* stage = reinterpret_cast<float4*>(smem);  // partial sums (split_piece order), while the ring is idle
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * KPS * PAIR_KB_BYTES);
+    // bars: full[STAGES] (pair leader), empty[STAGES], tfull, (unused), (unused), (unused), done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    float* off_s = reinterpret_cast<float*>(tmem_slot + 4);
+    float* bias_s = off_s + BN;
+    const Xch xch = carve_xch<BN>(bias_s + BN);
+    for (int i = threadIdx.x; i < 2 * BN; i += blockDim.x) xch.hist[i] = 0;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const uint32_t prank = rank & 1u, pair_leader = rank & ~1u;
+    const int pr = (int)(rank >> 1);  // this pair's share of each tile's k-blocks
+    const bool leader = prank == 0;
+    const int cluster = (int)blockIdx.x / (2 * splits), nclusters = (int)gridDim.x / (2 * splits);
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+    const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+    const uint32_t done_bar = smem_u32(bars + 2 * STAGES + 4);
+    const int num_kb = (d + BK - 1) / BK;
+    const int nslots = (num_kb + KPS - 1) / KPS;
+    const int kb_lo = (pr * nslots / splits) * KPS;
+    const int kb_hi = min(num_kb, ((pr + 1) * nslots / splits) * KPS);
+    const uint16_t pair_mask = (uint16_t)(3u << pair_leader);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+        mbar_init(tfull0, 1);
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(PairCfg::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < BN; i += blockDim.x) {
+        const float o = p.off != nullptr ? p.off[i] : 0.f;
+        const float b = p.bias != nullptr ? p.bias[i] : 0.f;
+        off_s[i] = p.bias_in_logits ? __fadd_rn(o, b) : o;
+        bias_s[i] = p.bias_in_logits ? 0.f : b;
+    }
+    fence_before();
+    cluster_sync();  // every CTA's barriers exist before any cross-CTA arrival
+    fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // The cluster walks its tiles one after another; every thread of every
+    // CTA takes the same iterations and meets the two cluster barriers of each
+    // (a role that has given up on a wait does nothing more but still meets
+    // them), so the accumulator and the staged partials are never overwritten
+    // while still being read.
+    uint32_t it = 0;   // ring slot sequence (producer and MMA issuer)
+    bool ok = true;    // this thread's waits have all succeeded
+    uint32_t local = 0;
+    for (int tp = cluster; tp < num_pairs; tp += nclusters, ++local) {
+        int epi_ok = 0;
+        if (warp == 0) {
+            // -------------------------------------------------------- producer (every CTA)
+            if (lane == 0 && ok) {
+                const int m0 = tp * 2 * BM + (int)prank * BM;
+                for (int kb = kb_lo; kb < kb_hi; kb += KPS, ++it) {
+                    const int nk = min(KPS, kb_hi - kb);
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!mbar_wait(empty0 + 8 * s, ph ^ 1, err)) { ok = false; break; }
+                    const uint32_t fb = map_to(full0 + 8 * s, pair_leader);
+                    if (leader) mbar_expect_tx(full0 + 8 * s, 2 * nk * PAIR_KB_BYTES);
+#pragma unroll
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        tma_load_2d_pair(smem_u32(sA + slot * A_KB_BYTES), &tmA, (kb + j) * BK, m0, fb);
+                        tma_load_2d_pair(smem_u32(sB + slot * A_KB_BYTES), &tmB, (kb + j) * BK, (int)prank * BM,
+                                         fb);
+                    }
+                }
+            }
+        } else if (warp == 1) {
+            // -------------------------------------------------------- MMA issuer (pair leaders)
+            if (leader && lane == 0 && ok) {
+                for (int kb = kb_lo; kb < kb_hi; kb += KPS, ++it) {
+                    const int nk = min(KPS, kb_hi - kb);
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!mbar_wait(full0 + 8 * s, ph, err)) { ok = false; break; }
+                    fence_after();
+#pragma unroll
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nk) break;
+                        const size_t slot = (size_t)s * KPS + j;
+                        const uint32_t a_addr = smem_u32(sA + slot * A_KB_BYTES);
+                        const uint32_t b_addr = smem_u32(sB + slot * A_KB_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16_pair(tmem_base, sdesc(a_addr + 32 * k), sdesc(b_addr + 32 * k), idesc_pair(),
+                                          (kb + j > kb_lo || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair_mask(empty0 + 8 * s, pair_mask);
+                }
+                if (ok) mma_commit_pair_mask(tfull0, pair_mask);
+            }
+        } else {
+            // -------------------------------------------------------- epilogue warps: the accumulator
+            const int q = warp & 3, h = (warp - 2) >> 2, row = q * 32 + lane, ew = warp - 2;
+            if (lane == 0) xch.agree[ew] = (ok && mbar_wait(tfull0, local & 1, err)) ? 1 : 0;
+            epi_sync();
+            epi_ok = 1;
+#pragma unroll
+            for (int w = 0; w < EPI_WARPS; ++w) epi_ok &= xch.agree[w];
+            epi_sync();  // every warp has read the verdicts before the next tile's are written
+            if (!epi_ok) ok = false;
+            fence_after();
+            if (epi_ok && pr != 0) {
+                // this pair's partial sums into the idle ring (rows padded against bank conflicts)
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+                for (int cc = 0; cc < NCH; ++cc) {
+                    const int c = h * NCH + cc;
+                    float v[32];
+                    tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq)
+                        stage[split_piece(c, qq, row)] =
+                            make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]);
+                }
+            }
+        }
+
+        // every partial of this tile is staged before pair 0 reads it
+        fence_before();
+        __syncthreads();
+        cluster_sync();
+        fence_after();
+
+        if (warp >= 2 && pr == 0 && epi_ok) {
+            const int q = warp & 3, h = (warp - 2) >> 2, row = q * 32 + lane;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+            // the other pairs' partial sums, in pair order, added into this CTA's accumulator
+#pragma unroll 1
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int c = h * NCH + cc;
+                float v[32];
+                tmem_ld32(taddr + 32 * c, v);
+                const uint32_t src = smem_u32(stage + split_piece(c, 0, row));
+                // two pairs' pieces in flight at once, added in pair order
+                for (int p2 = 1; p2 < splits; p2 += 2) {
+                    const bool two = p2 + 1 < splits;
+                    const uint32_t peer_a = map_to(src, 2u * (uint32_t)p2 + prank);
+                    const uint32_t peer_b = map_to(src, 2u * (uint32_t)(two ? p2 + 1 : p2) + prank);
+                    float4 fa[8], fb[8];
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) {
+                        fa[qq] = ld_dsmem_f4(peer_a + 16u * 128u * (uint32_t)qq);
+                        fb[qq] = ld_dsmem_f4(peer_b + 16u * 128u * (uint32_t)qq);
+                    }
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) {
+                        v[4 * qq] += fa[qq].x;
+                        v[4 * qq + 1] += fa[qq].y;
+                        v[4 * qq + 2] += fa[qq].z;
+                        v[4 * qq + 3] += fa[qq].w;
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq) {
+                            v[4 * qq] += fb[qq].x;
+                            v[4 * qq + 1] += fb[qq].y;
+                            v[4 * qq + 2] += fb[qq].z;
+                            v[4 * qq + 3] += fb[qq].w;
+                        }
+                    }
+                }
+                tmem_st32(taddr + 32 * c, v);
+            }
+            const int64_t grow = (int64_t)tp * 2 * BM + (int64_t)prank * BM + row;
+            epilogue_row<BN, FUSED>(p, taddr, row, h, grow, off_s, bias_s, xch);
+            if (FUSED && p.tile_counts != nullptr) flush_tile_hist<BN>(p, xch, (int64_t)tp * 2 + prank);
+        }
+
+        // pair 0 has read every partial and finished with the accumulators
+        // before the next tile's loads and MMAs reuse the ring and TMEM
+        fence_before();
+        __syncthreads();
+        cluster_sync();
+        fence_after();
+    }
+
+    // the MMA issuers' MMAs are complete before TMEM is freed
+    if (warp == 1 && leader && lane == 0) {
+        mma_commit_pair_local(done_bar);
+        mbar_wait(done_bar, 0, err, /*watch=*/false);
+    }
+    fence_before();
+    __syncthreads();
+    cluster_sync();
+    fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(PairCfg::TMEM_COLS)
+                     : "memory");
+    }
+}
+
 }  // namespace tc
 
 // ---------------------------------------------------------------------------
@@ -894,17 +1160,91 @@ bool gate_tc_can_fuse(int N, int K, int fn, int n_groups, int group_topn) {
     return fn == MOE_SIGMOID && N / n_groups == 32 && group_topn >= 1 && group_topn <= 2;
 }
 
+// Launch configuration of the split-K pair kernel: one tile per cluster of
+// 2 * splits CTAs.
+static cudaLaunchConfig_t split_config(int num_pairs, int splits, size_t smem, cudaStream_t st,
+                                       cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(num_pairs * 2 * splits), 1, 1);
+    cfg.blockDim = dim3(tc::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)(2 * splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// How many CTA pairs share each tile's k-blocks, from the batch shape and the
+// device alone (so that the result does not depend on an SM budget): 1 unless
+// at least half of the device's CTA pairs would otherwise sit idle; at most 4
+// (clusters of 8 CTAs), at least two ring slots of k-blocks per pair, and no
+// more than lets one cluster per tile be resident at once (on a B200 with this
+// kernel's shared memory: 74 clusters of 2 CTAs, 33 of 4, 22 of 6, 15 of 8).
+// MOE_GATE_SPLIT=0 turns it off.
+static int split_resident(int splits, bool fused, size_t smem) {
+    static int resident[2][5] = {};  // [fused][splits]: clusters that fit at once (-1: none)
+    int& r = resident[fused ? 1 : 0][splits];
+    if (r == 0) {
+        auto kern = fused ? tc::gate_tc_split_kernel<true> : tc::gate_tc_split_kernel<false>;
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = split_config(1, splits, smem, nullptr, attr);
+        int n = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
+            n = 0;
+        r = n > 0 ? n : -1;
+    }
+    return r;
+}
+
+static int choose_splits(int num_pairs, int num_kb, bool fused, size_t smem) {
+    const char* env = getenv("MOE_GATE_SPLIT");
+    if (env != nullptr && env[0] == '0') return 1;
+    const int device_pairs = moe_host::sm_count() / 2;
+    if (num_pairs < 1 || 2 * num_pairs > device_pairs) return 1;
+    const int nslots = (num_kb + tc::PAIR_KPS - 1) / tc::PAIR_KPS;
+    int s = device_pairs / num_pairs;
+    if (s > 4) s = 4;
+    while (s >= 2 && nslots < 2 * s) --s;
+    while (s >= 2 && split_resident(s, fused, smem) < num_pairs) --s;  // every tile's cluster at once
+    return s < 2 ? 1 : s;
+}
+
 static cudaError_t launch_pair(const void* x, const void* W, int T, int d, const tc::Epi& p, int32_t* err,
                                int max_ctas, cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, x, T, d, tc::BM) || !make_map(&mb, W, 256, d, tc::BM)) return cudaErrorInvalidValue;
     const size_t smem = tc::PairCfg::SMEM_BYTES;
-    auto kern = p.fused ? tc::gate_tc_pair_kernel<true> : tc::gate_tc_pair_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int num_pairs = (T + 2 * tc::BM - 1) / (2 * tc::BM);
     int clusters = moe_host::sm_count() / 2;
     if (max_ctas > 0 && clusters > max_ctas / 2) clusters = max_ctas / 2;
+    int splits = choose_splits(num_pairs, (d + tc::BK - 1) / tc::BK, p.fused != 0, smem);
+    if (splits > 1 && max_ctas > 0 && max_ctas < 2 * splits) splits = 1;  // a budget below one cluster
+    if (splits > 1) {
+        // clusters: one per tile, within the SM budget and what fits at once;
+        // each walks its tiles in turn, so the result is the same for any count
+        int ncl = num_pairs;
+        if (max_ctas > 0 && ncl > max_ctas / (2 * splits)) ncl = max_ctas / (2 * splits);
+        const int res = split_resident(splits, p.fused != 0, smem);
+        if (ncl > res) ncl = res;
+        if (ncl < 1) ncl = 1;
+        auto skern = p.fused ? tc::gate_tc_split_kernel<true> : tc::gate_tc_split_kernel<false>;
+        cudaError_t e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = split_config(ncl, splits, smem, st, attr);
+        e = cudaLaunchKernelEx(&cfg, skern, ma, mb, d, p, err, num_pairs, splits);
+        moe_host::note_launch();
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    auto kern = p.fused ? tc::gate_tc_pair_kernel<true> : tc::gate_tc_pair_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     if (clusters > num_pairs) clusters = num_pairs;
     if (clusters < 1) clusters = 1;
     kern<<<2 * clusters, tc::THREADS, smem, st>>>(ma, mb, d, p, err, num_pairs);

@@ -153,3 +153,26 @@ def test_gate_one_sm_and_pair_agree(pair, monkeypatch):
     assert lib().moe_workspace_status(ws) == 0
     ref = inp["x"].cuda().float() @ inp["W"].cuda().float().t()
     assert torch.allclose(s, torch.sigmoid(ref), rtol=1e-3, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,d", [(4096, 7168), (300, 7168), (700, 936), (1, 2048)])
+def test_gate_split_k_matches_unsplit(monkeypatch, T, d):
+    """With fewer 256-token tiles than half the CTA pairs the pair kernel
+    splits each tile's k-blocks over up to four pairs of one cluster and adds
+    their partial sums in pair order.  The scores equal the unsplit kernel's
+    up to fp32 summation order, and repeated runs are bit-identical (the
+    order of the additions does not depend on timing)."""
+    wl = W.WORKLOADS["v3_router"].with_(T=T, d=d)
+    inp = W.make_inputs(wl, seed=T + d)
+    x, Wg, b = inp["x"].cuda(), inp["W"].cuda(), inp["bias"].cuda()
+    s1, i1, w1, ws1 = route_gpu(wl, x, Wg, None, b)
+    s2, i2, w2, ws2 = route_gpu(wl, x, Wg, None, b)
+    monkeypatch.setenv("MOE_GATE_SPLIT", "0")
+    s0, _, _, ws0 = route_gpu(wl, x, Wg, None, b)
+    torch.cuda.synchronize()
+    for ws in (ws0, ws1, ws2):
+        assert lib().moe_workspace_status(ws) == 0
+    assert torch.equal(s1, s2) and torch.equal(i1, i2) and torch.equal(w1, w2)
+    assert torch.allclose(s1, s0, rtol=1e-4, atol=1e-6)
+    ref = torch.sigmoid(x.float() @ Wg.float().t())
+    assert torch.allclose(s1, ref, rtol=1e-3, atol=1e-6)
