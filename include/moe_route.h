@@ -74,7 +74,10 @@ typedef struct {
     int32_t gate_max_ctas; /* at most this many CTAs (SMs) for the tensor-core gate GEMM,
                               0 = all SMs; a smaller budget leaves SMs to work running
                               beside it on another stream (e.g. the previous batch's
-                              dispatch) */
+                              dispatch).  The scores do not depend on the budget, except
+                              that a budget below 8 CTAs turns off the small-batch split
+                              of the k-blocks over CTA pairs, which changes the fp32
+                              summation order */
 } moe_route_cfg;
 
 /* Load statistics of one histogram, written to device memory.
