@@ -75,9 +75,9 @@ typedef struct {
                               0 = all SMs; a smaller budget leaves SMs to work running
                               beside it on another stream (e.g. the previous batch's
                               dispatch).  The scores do not depend on the budget, except
-                              that a budget below 8 CTAs turns off the small-batch split
-                              of the k-blocks over CTA pairs, which changes the fp32
-                              summation order */
+                              that a budget smaller than one cluster of the small-batch
+                              split of the k-blocks over CTA pairs (4 to 8 CTAs) turns
+                              the split off, which changes the fp32 summation order */
 } moe_route_cfg;
 
 /* Load statistics of one histogram, written to device memory.
