@@ -77,6 +77,16 @@ def test_gate_tc_against_oracle(orc, name, T, d):
     _run_and_check(orc, W.WORKLOADS[name], T, d, seed=T + d)
 
 
+def test_gate_tc_n256_softmax_small_batch(orc):
+    """N = 256 with the row softmax, at batch sizes where the pair kernel
+    splits each tile's k-blocks over several CTA pairs (the softmax epilogue
+    then runs on the added partial sums) and where it does not."""
+    wl = W.Workload("n256sm", 0, 0, 0, 256, 8, fn=0, scale=1.0, has_bias=True)
+    _run_and_check(orc, wl, 600, 2048, seed=11)   # 3 tiles: split over 4 pairs
+    _run_and_check(orc, wl, 97, 1000, seed=12)    # 1 ragged tile, 16 k-blocks: split
+    _run_and_check(orc, wl, 700, 128, seed=13)    # 2 k-blocks: too few to split
+
+
 def test_gate_tc_n64_sigmoid(orc):
     wl = W.Workload("n64", 0, 0, 0, 64, 6, fn=1, n_groups=4, topk_groups=2, scale=1.0, has_bias=True)
     _run_and_check(orc, wl, 700, 512, seed=3)
