@@ -269,6 +269,85 @@ __device__ __forceinline__ void store_chunk_staged(const Epi& p, int64_t grow, i
     }
 }
 
+// One group (every expert a candidate): the fused selection over this half's
+// columns.  Pass A computes each 8-column piece's values and keys (writing the
+// scores when they are wanted) and keeps the r = ceil(K/2) largest of the
+// pieces' second-largest keys; the halves exchange theirs, and theta, the r-th
+// largest of them over the whole row, bounds the K-th best key from below (at
+// least r pieces hold two keys >= theta).  Pass B offers, from the same values,
+// only the keys >= theta, in rounds of one per lane (lanes are rows with
+// different survivors).  `value` turns a raw accumulator column into the score.
+template <int BN, typename F>
+__device__ __forceinline__ void one_group_select(const Epi& p, uint32_t taddr, int row, int h, int c_lo, float* srow,
+                                                 const float* bias_s, float* xg, Top8& top, F value) {
+    constexpr int NQ = 4 * (BN / 64);  // 8-column pieces in a half row
+    const int r = (p.K + 1) >> 1;
+    float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // descending
+#pragma unroll 1
+    for (int q = 0; q < NQ; ++q) {
+        const int col0 = 32 * c_lo + 8 * q;
+        float v8[8];
+        tmem_ld8(taddr + col0, v8);
+        float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v8[i] = value(v8[i], col0 + i);
+            const float k = __fadd_rn(v8[i], bias_s[col0 + i]);
+            t2 = fmaxf(t2, fminf(t1, k));
+            t1 = fmaxf(t1, k);
+        }
+        if (srow) store8(srow + col0, v8);
+        float x = t2;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float hi = fmaxf(b4[j], x);
+            x = fminf(b4[j], x);
+            b4[j] = hi;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xg[row * 8 + h * 4 + j] = b4[j];
+    epi_sync();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float x = xg[row * 8 + (1 - h) * 4 + j];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const float hi = fmaxf(b4[jj], x);
+            x = fminf(b4[jj], x);
+            b4[jj] = hi;
+        }
+    }
+    float theta = b4[0];
+#pragma unroll
+    for (int j = 1; j < 4; ++j)
+        if (j < r) theta = b4[j];
+#pragma unroll 1
+    for (int q = 0; q < NQ; ++q) {
+        const int col0 = 32 * c_lo + 8 * q;
+        float v8[8], k8[8];
+        tmem_ld8(taddr + col0, v8);
+        unsigned m = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v8[i] = value(v8[i], col0 + i);
+            k8[i] = __fadd_rn(v8[i], bias_s[col0 + i]);
+            if (!(k8[i] < theta)) m |= 1u << i;  // a NaN key is offered
+        }
+        while (__any_sync(0xffffffffu, m != 0)) {
+            if (m != 0) {
+                const int i = __ffs(m) - 1;
+                m &= m - 1;
+                float kk = k8[0], sv = v8[0];
+#pragma unroll
+                for (int j = 1; j < 8; ++j)
+                    if (i == j) { kk = k8[j]; sv = v8[j]; }
+                top.offer(kk, col0 + i, sv);
+            }
+        }
+    }
+}
+
 // One token row (this thread's TMEM lane) of one finished tile.  The two
 // warps of a lane quarter split the columns: half h owns chunks
 // [h*NC/2, (h+1)*NC/2) of 32 columns.  Softmax exchanges the row max and sum;
@@ -296,7 +375,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
+                    v[i] = sigmoid_f(__fadd_rn(v[i], off_s[32 * c + i]));
                     const float key = __fadd_rn(v[i], bias_s[32 * c + i]);
                     if (key > t1) { t2 = t1; t1 = key; } else if (key > t2) { t2 = key; }
                 }
@@ -340,7 +419,7 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int col = 32 * c + 8 * q + i;
-                        v8[i] = sigmoid_f(v8[i] + off_s[col]);
+                        v8[i] = sigmoid_f(__fadd_rn(v8[i], off_s[col]));
                         k8[i] = __fadd_rn(v8[i], bias_s[col]);
                         if (kc && !(k8[i] < t0)) m |= 1u << i;  // a NaN key is offered, as without the bound
                     }
@@ -359,25 +438,15 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
                 }
             }
         } else if constexpr (FUSED) {
-#pragma unroll 1
-            for (int q = 0; q < 4 * NCH; ++q) {
-                const int col0 = 32 * c_lo + 8 * q;
-                float v8[8];
-                tmem_ld8(taddr + col0, v8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    v8[i] = sigmoid_f(v8[i] + off_s[col0 + i]);
-                    top.offer(__fadd_rn(v8[i], bias_s[col0 + i]), col0 + i, v8[i]);
-                }
-                if (srow) store8(srow + col0, v8);
-            }
+            one_group_select<BN>(p, taddr, row, h, c_lo, srow, bias_s, x.gs, top,
+                                 [&](float a, int col) { return sigmoid_f(__fadd_rn(a, off_s[col])); });
         } else {
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
                 tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = sigmoid_f(v[i] + off_s[32 * c + i]);
+                for (int i = 0; i < 32; ++i) v[i] = sigmoid_f(__fadd_rn(v[i], off_s[32 * c + i]));
                 if (p.scores != nullptr) store_chunk_staged<BN>(p, grow, c, v, x.stage + warp_in_epi * (32 * 20), lane);
             }
         }
@@ -400,31 +469,22 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
             const int c = c_lo + cc;
             tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum += expf(v[i] + off_s[32 * c + i] - m);
+            for (int i = 0; i < 32; ++i) sum += expf(__fsub_rn(__fadd_rn(v[i], off_s[32 * c + i]), m));
         }
         x.red[(h * 2 + 1) * BM + row] = sum;
         epi_sync();
         const float inv = 1.f / (x.red[1 * BM + row] + x.red[3 * BM + row]);
         if constexpr (FUSED) {
-#pragma unroll 1
-            for (int q = 0; q < 4 * NCH; ++q) {
-                const int col0 = 32 * c_lo + 8 * q;
-                float v8[8];
-                tmem_ld8(taddr + col0, v8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    v8[i] = expf(v8[i] + off_s[col0 + i] - m) * inv;
-                    top.offer(__fadd_rn(v8[i], bias_s[col0 + i]), col0 + i, v8[i]);
-                }
-                if (srow) store8(srow + col0, v8);
-            }
+            one_group_select<BN>(p, taddr, row, h, c_lo, srow, bias_s, x.gs, top, [&](float a, int col) {
+                return __fmul_rn(expf(__fsub_rn(__fadd_rn(a, off_s[col]), m)), inv);
+            });
         } else {
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
                 tmem_ld32(taddr + 32 * c, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = expf(v[i] + off_s[32 * c + i] - m) * inv;
+                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(expf(__fsub_rn(__fadd_rn(v[i], off_s[32 * c + i]), m)), inv);
                 if (p.scores != nullptr) store_chunk_staged<BN>(p, grow, c, v, x.stage + warp_in_epi * (32 * 20), lane);
             }
         }

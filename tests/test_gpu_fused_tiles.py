@@ -173,3 +173,31 @@ def test_route_tiles_with_ties_match_oracle(orc, monkeypatch, kind):
     assert np.array_equal(to_np(tiles), _tile_hist_ref(ri, wl.N))
     if kind == "zero_gate":
         assert np.array_equal(ri, np.broadcast_to(np.arange(wl.K, dtype=ri.dtype), ri.shape))
+
+
+@pytest.mark.parametrize("kind", ["softmax_n128", "softmax_zero_gate", "sigmoid_one_group", "softmax_twins"])
+def test_route_tiles_one_group_match_oracle(orc, monkeypatch, kind):
+    """One group (every expert a candidate): the epilogue's bound comes from
+    the 8-column pieces' second-largest keys of both row halves.  Random
+    scores, a zero gate (every key equal: the lowest experts win) and experts
+    sharing their gate rows in pairs (ties at and around the bound)."""
+    if kind == "sigmoid_one_group":
+        wl = W.Workload("sig1", 0, 900, 1024, 256, 8, fn=1, scale=2.5, has_bias=True)
+    else:
+        wl = W.Workload("sm128", 0, 900, 1024, 128, 8, fn=0, scale=1.0, has_bias=kind == "softmax_twins")
+    inp = W.make_inputs(wl, device="cuda", seed=43)
+    if kind == "softmax_zero_gate":
+        inp["W"] = torch.zeros_like(inp["W"])
+    if kind == "softmax_twins":
+        src = torch.arange(wl.N, device="cuda") // 2 * 2
+        inp["W"] = inp["W"][src].contiguous()
+        inp["bias"] = inp["bias"][src].contiguous()
+    idx, w, tiles, _ = _fused(wl, inp)
+    s = _scores_only(wl, inp, monkeypatch)
+    b = inp["bias"].cpu().numpy() if inp["bias"] is not None else None
+    ri, rw = orc.select(to_np(s), b, wl.K, wl.n_groups, wl.topk_groups, wl.group_topn, wl.renorm, wl.scale)
+    assert np.array_equal(to_np(idx), ri)
+    assert np.array_equal(to_np(w), rw)
+    assert np.array_equal(to_np(tiles), _tile_hist_ref(ri, wl.N))
+    if kind == "softmax_zero_gate":
+        assert np.array_equal(ri, np.broadcast_to(np.arange(wl.K, dtype=ri.dtype), ri.shape))
