@@ -27,6 +27,7 @@
 // Every barrier wait is bounded: on expiry the kernel records the error in
 // the workspace, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <math.h>
 #include <stdlib.h>
 
@@ -367,17 +368,31 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
     top.init();
     if (p.fn == MOE_SIGMOID) {
         if (FUSED && p.n_groups > 1) {
-            // one expert group per 32-column chunk: group score = sum of its top-n keys
+            // one expert group per 32-column chunk: group score = sum of its top-n
+            // keys; each 8-column piece's second-largest key also goes to shared
+            // memory (rounded down to half precision: still a lower bound) for
+            // the bound below, in the merge lists' space (idle until the merge)
+            __half* piece_t2 = reinterpret_cast<__half*>(x.lk) + row * 32;
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
                 tmem_ld32(taddr + 32 * c, v);
-                float t1 = -INFINITY, t2 = -INFINITY;
+                float a1[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, a2[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     v[i] = sigmoid_f(__fadd_rn(v[i], off_s[32 * c + i]));
                     const float key = __fadd_rn(v[i], bias_s[32 * c + i]);
-                    if (key > t1) { t2 = t1; t1 = key; } else if (key > t2) { t2 = key; }
+                    a2[i >> 3] = fmaxf(a2[i >> 3], fminf(a1[i >> 3], key));  // a NaN key enters none
+                    a1[i >> 3] = fmaxf(a1[i >> 3], key);
+                }
+                float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc) {
+                    t2 = fmaxf(t2, fminf(t1, a1[pc]));
+                    t1 = fmaxf(t1, a1[pc]);
+                    t2 = fmaxf(t2, fminf(t1, a2[pc]));
+                    t1 = fmaxf(t1, a2[pc]);
+                    piece_t2[4 * c + pc] = __float2half_rd(a2[pc]);
                 }
                 x.gs[row * 8 + c] = p.group_topn == 1 ? t1 : __fadd_rn(t1, t2);
                 x.gt2[row * 8 + c] = t2;
@@ -406,6 +421,34 @@ __device__ __forceinline__ void epilogue_row(const Epi& p, uint32_t taddr, int r
             for (int c = 0; c < NC; ++c)
                 if ((keep >> c) & 1u) t0 = fminf(t0, x.gt2[row * 8 + c]);
             if (2 * p.topk_groups < p.K || !(t0 < INFINITY)) t0 = -INFINITY;
+            // A second bound, tighter when one group holds most of the best keys:
+            // the ceil(K/2)-th largest second-largest key over the kept groups'
+            // 8-column pieces (at least that many pieces hold two keys at or
+            // above it).  Both bound the K-th best key, so their maximum does.
+            {
+                float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // descending
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    if (!((keep >> c) & 1u)) continue;
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc) {
+                        float xv = __half2float(piece_t2[4 * c + pc]);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float hi = fmaxf(b4[j], xv);
+                            xv = fminf(b4[j], xv);
+                            b4[j] = hi;
+                        }
+                    }
+                }
+                const int r = (p.K + 1) >> 1;
+                float thp = b4[0];
+#pragma unroll
+                for (int j = 1; j < 4; ++j)
+                    if (j < r) thp = b4[j];
+                t0 = fmaxf(t0, thp);
+            }
+            epi_sync();  // every row's pieces are read before the merge lists reuse their space
 #pragma unroll 1
             for (int cc = 0; cc < NCH; ++cc) {
                 const int c = c_lo + cc;
