@@ -186,3 +186,25 @@ def test_gate_split_k_matches_unsplit(monkeypatch, T, d):
     assert torch.allclose(s1, s0, rtol=1e-4, atol=1e-6)
     ref = torch.sigmoid(x.float() @ Wg.float().t())
     assert torch.allclose(s1, ref, rtol=1e-3, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,d", [(255, 7168), (256, 640), (257, 704), (511, 1088), (2049, 2048), (3841, 1024),
+                                 (3840, 7168), (4097, 4096), (7000, 1536), (9472, 1024), (9473, 1024)])
+def test_gate_split_k_sweep(monkeypatch, T, d):
+    """Batch sizes around the thresholds of the small-batch split (tile
+    edges; S = 4, 3, 2 pairs; the largest batch that still splits and the
+    first that does not) and k-block counts that do not divide evenly:
+    scores equal the unsplit kernel's up to fp32 summation order, and a
+    second run gives bit-identical scores and choices (with the selection in
+    its own kernel and in the epilogue)."""
+    wl = W.WORKLOADS["v3_router"].with_(T=T, d=d)
+    inp = W.make_inputs(wl, seed=T * 7 + d)
+    x, Wg, b = inp["x"].cuda(), inp["W"].cuda(), inp["bias"].cuda()
+    s1, i1, w1, ws1 = route_gpu(wl, x, Wg, None, b)
+    s2, i2, _, _ = route_gpu(wl, x, Wg, None, b)
+    monkeypatch.setenv("MOE_GATE_SPLIT", "0")
+    s0, _, _, ws0 = route_gpu(wl, x, Wg, None, b)
+    torch.cuda.synchronize()
+    assert lib().moe_workspace_status(ws1) == 0 and lib().moe_workspace_status(ws0) == 0
+    assert torch.equal(s1, s2) and torch.equal(i1, i2)
+    assert torch.allclose(s1, s0, rtol=1e-4, atol=1e-6)
